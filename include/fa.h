@@ -1,0 +1,144 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact IO-aware scaled-dot-product attention on
+ * one NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  O = softmax(scale * Q K^T + causal mask) V, the plain
+ * definition of attention ("FlashAttention 심층 분석", section 1), evaluated
+ * tile by tile with the online softmax of section 3 of the same page (running
+ * max m, running sum l, rescaling of O) so that the N x N score matrix never
+ * reaches HBM.  The forward pass keeps one fp32 log-sum-exp per query row
+ * (smithlab guide to FlashAttention versions and training cost, memory table) and the
+ * backward pass recomputes P from it (same analysis page, section 4).  One-token
+ * decode splits the key axis and merges the splits by log-sum-exp (analysis
+ * page, "Flash-Decoding").  GQA is expressed by the KV-head count, with no K/V
+ * copies, and causal masking is a flag (smithlab guide, adoption checklist).
+ *
+ * Conventions shared by every entry point:
+ *  - Layout "BSHD", contiguous, d innermost:
+ *      q, o, dout, dq : [B, Nq, Hq, d]      k, v, dk, dv : [B, Nk, Hkv, d]
+ *      lse, D         : [B, Hq, Nq] fp32    decode caches : [B, Nk_max, Hkv, d]
+ *  - Element type of q/k/v/o/dout/dq/dk/dv: fa_dtype (IEEE fp16 or bf16).
+ *  - LSE is the natural-log log-sum-exp of the scaled, masked scores of a row.
+ *  - Causal keeps key j for query i iff j <= i + (Nk - Nq) (bottom-right
+ *    alignment; the lower triangle when Nq == Nk).  causal requires Nq <= Nk.
+ *  - GQA: Hq % Hkv == 0; query head h reads KV head h / (Hq / Hkv).
+ *  - d must be 64 or 128 (FA_ERR_UNSUPPORTED otherwise).  Nq, Nk >= 1, any
+ *    value (ragged tails are masked inside the kernels).
+ *  - Every pointer is a DEVICE pointer, 16-byte aligned (FA_ERR_ALIGN).  The
+ *    caller owns and allocates every buffer, workspaces included; the library
+ *    never allocates device memory and keeps no per-call state.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  The return value reports argument validation (checked
+ *    before anything is launched) and launch errors only.  Errors raised by a
+ *    running kernel (a bounded wait that ran out, see fa_get_device_status)
+ *    are recorded in a device status word.
+ *  - Outputs are overwritten, never accumulated into.  Results are
+ *    deterministic: two calls on the same inputs give bitwise-equal outputs.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID = -1,     /* null pointer, bad size, Hq % Hkv != 0, causal with Nq > Nk */
+  FA_ERR_UNSUPPORTED = -2, /* d not in {64, 128}, unknown dtype, size beyond a stated limit */
+  FA_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned */
+  FA_ERR_CUDA = -4,        /* a CUDA runtime/driver call or a launch failed */
+  FA_ERR_TIMEOUT = -5      /* a kernel's bounded wait ran out (device status word) */
+} fa_status;
+
+typedef enum { FA_FP16 = 0, FA_BF16 = 1 } fa_dtype;
+
+/* A cudaStream_t passed as an opaque pointer (keeps this header free of CUDA includes). */
+typedef void* fa_stream_t;
+
+/*
+ * Forward pass.  Writes o [B,Nq,Hq,d] (dtype dt) and lse [B,Hq,Nq] (fp32).
+ * Source: "FlashAttention 심층 분석", sections 1 and 3 (definition; tiling and
+ * online softmax fused into one kernel: scale, mask, softmax, PV).
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                 fa_dtype dt, fa_stream_t stream);
+
+/* Bytes of workspace fa_bwd needs: the fp32 row term D [B,Hq,Nq]. */
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq);
+
+/*
+ * Backward pass.  Given q, k, v, the forward output o, the upstream gradient
+ * dout and the forward lse, writes dq, dk, dv (dtype dt), each overwritten.
+ * P is recomputed from lse ("FlashAttention 심층 분석", section 4); the
+ * gradients are the chain rule of the definition:
+ *   D_i = sum_c dO_ic O_ic,  dS = P * (dO V^T - D),
+ *   dV = P^T dO,  dQ = scale dS K,  dK = scale dS^T Q,
+ * with dK, dV of a KV head summed over its Hq/Hkv query heads.  `workspace`
+ * must hold fa_bwd_workspace_bytes(B, Hq, Nq) bytes (device, 16-byte aligned).
+ * No atomics: dK/dV and dQ come from separate kernels, so the result is
+ * bitwise reproducible (the deterministic mode of the smithlab guide's
+ * recommendation table).
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                 int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                 fa_dtype dt, fa_stream_t stream);
+
+/*
+ * Suggested number of key splits for fa_decode_splitkv: enough (b, h_kv, split)
+ * units to fill `num_sms` SMs several times over (num_sms <= 0: query the
+ * current device).  Always >= 1 and <= ceil(Nk_max / 64).
+ */
+int fa_decode_num_splits(int B, int Hkv, int Nk_max, int d, int num_sms);
+
+/* Bytes of the split partials: O_s fp32 [B,Hq,num_splits,d] + LSE_s fp32 [B,Hq,num_splits]. */
+size_t fa_decode_workspace_bytes(int B, int Hq, int num_splits, int d);
+
+/*
+ * Split-KV decode, partial pass ("FlashAttention 심층 분석", Flash-Decoding).
+ * q [B,1,Hq,d]; k_cache, v_cache [B,Nk_max,Hkv,d]; seqlens_k: DEVICE int32 [B],
+ * 0 <= seqlens_k[b] <= Nk_max (values outside are clamped into that range).
+ * Split s of sequence b covers keys [s*C, min((s+1)*C, seqlens_k[b])) with
+ * C = fa_decode_chunk(Nk_max, num_splits); each split writes its normalised
+ * partial output O_s and LSE_s into `workspace` (an empty split writes O_s = 0,
+ * LSE_s = -inf).  Non-causal: the query is the newest token.
+ */
+fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
+                            const int* seqlens_k, int B, int Hq, int Hkv, int Nk_max, int d,
+                            float scale, int num_splits, void* workspace, fa_dtype dt,
+                            fa_stream_t stream);
+
+/*
+ * Split-KV decode, combine pass: LSE = ln sum_s exp(LSE_s) and
+ * O = sum_s exp(LSE_s - LSE) O_s, cast to dt.  o [B,1,Hq,d]; lse [B,Hq,1] fp32.
+ * A sequence with seqlens_k[b] == 0 gets O = 0 and LSE = -inf.
+ */
+fa_status fa_decode_combine(const void* workspace, void* o, float* lse, const int* seqlens_k,
+                            int B, int Hq, int num_splits, int d, fa_dtype dt,
+                            fa_stream_t stream);
+
+/* Keys per split used by fa_decode_splitkv: ceil(Nk_max / num_splits) rounded up to 64. */
+int fa_decode_chunk(int Nk_max, int num_splits);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word that the
+ * kernels set when a bounded wait runs out (FA_ERR_TIMEOUT) or a device-side
+ * check fails.  Returns FA_OK when no kernel reported an error.
+ */
+fa_status fa_get_device_status(fa_stream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* fa_status_string(fa_status s);
+
+/* Library version, for the binding's sanity check. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */
