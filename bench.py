@@ -1,0 +1,493 @@
+#!/usr/bin/env python
+"""Throughput of exact IO-aware attention on B200, one JSON line on stdout.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one GQA training step of attention: forward then backward on
+B=1, Hq=32, Hkv=8, N=8192, d=128, causal, bf16 (fwd kernel, then the three
+backward launches: D preprocess, dK/dV, dQ).  ``value`` is whole-job
+fwd+bwd TFLOP/s with the inputs resident in HBM, FLOPs counted as
+4 B Hq Nq Nk d / 2 for the causal forward and 2.5x that for the backward.
+The split-KV decode workload (B=64, Hq=32, Hkv=8, Nk_max=32768 with a ragged
+second half, d=128, bf16) is timed in the same run and reported as HBM GB/s
+under ``decode``.  Every input is synthetic and seeded; each step touches
+more bytes than the 126 MB L2 holds, so no explicit flush is done.
+
+Under torchrun (N > 1) every rank runs the same per-GPU workload on its own
+GPU (weak scaling; the work shards by (b, h_kv) with no data exchange), the
+timed region is bracketed by barriers, and the max over ranks is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd bf16 TFLOP/s & % of B200 dense peak; decode HBM GB/s"
+DENSE_BF16_DATASHEET_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def attn_flops(B, Hq, Nq, Nk, d, causal):
+    """Nominal forward FLOPs: two matmuls of 2 FLOPs per multiply-add, halved when causal."""
+    f = 4.0 * B * Hq * Nq * Nk * d
+    return f * 0.5 if causal else f
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's
+    source has not changed since the counters were taken (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        t = json.load(f).get(kernel)
+    if not t:
+        return None
+    try:
+        if source_hash(t["sources"]) != t["source_hash"]:
+            return None
+    except OSError:
+        return None
+    return t["dram_bytes_per_launch"]
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting", 0x10: "sync_boost",
+    }
+
+    def __init__(self, index, period=0.01):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period, self._stop = period, threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = get_r(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_init(torch):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(torch, world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(torch, world, x: float) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+
+    import exact_io_aware_80_b200 as fa
+    import workloads
+    from exact_io_aware_80_b200 import _lib
+
+    world, rank, local = dist_init(torch)
+    dev = torch.device("cuda", local)
+    _lib.load()
+    peaks, peaks_kind = load_peaks()
+
+    w = workloads.get(3)
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.Nq, w.d
+    q, k, v, do = workloads.workload_inputs(w, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, N, device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_workspace_bytes(B, Hq, N), device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    dt = _lib.FA_BF16
+    ptrs = [t.data_ptr() for t in (q, k, v, o, do, lse, dq, dk, dv, ws)]
+    bargs = ptrs + [B, Hq, Hkv, N, N, d, 1, w.scale, dt, sh]
+
+    def fwd():
+        _lib.fa_fwd(ptrs[0], ptrs[1], ptrs[2], ptrs[3], ptrs[5], B, Hq, Hkv, N, N, d, 1, w.scale, dt, sh)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        fwd()
+        if ev:
+            ev[1].record(stream)
+        _lib.fa_bwd_preprocess(*bargs)
+        if ev:
+            ev[2].record(stream)
+        _lib.fa_bwd_dkdv(*bargs)
+        if ev:
+            ev[3].record(stream)
+        _lib.fa_bwd_dq(*bargs)
+        if ev:
+            ev[4].record(stream)
+
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize(dev)
+    if fa.device_status() != 0:
+        raise RuntimeError("kernel status word set during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(torch, world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for i in range(K):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(torch, world)
+    ms = t0.elapsed_time(t1)
+    ms_max = max_over_ranks(torch, world, ms)
+    if fa.device_status() != 0:
+        raise RuntimeError("kernel status word set during the timed region")
+    per = {name: statistics.fmean(e[j].elapsed_time(e[j + 1]) for e in evs)
+           for j, name in enumerate(("fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"))}
+
+    F = attn_flops(B, Hq, N, N, d, True)
+    ms_step = ms_max / K
+    value = world * (F * 3.5) / (ms_step * 1e-3) / 1e12
+    fwd_tflops = F / (per["fwd"] * 1e-3) / 1e12
+    bwd_ms = per["bwd_preprocess"] + per["bwd_dkdv"] + per["bwd_dq"]
+    bwd_tflops = 2.5 * F / (bwd_ms * 1e-3) / 1e12
+
+    # roofline of the kernel with the largest share of the step
+    timed_region_s = ms / 1e3
+    peak_key = "bf16_tflops_sustained" if timed_region_s >= 2.0 else "bf16_tflops"
+    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    # FLOPs each kernel must execute: fwd 2 GEMMs (F), dK/dV 4 GEMMs (2F), dQ 3 GEMMs (1.5F)
+    kflops = {"fwd": F, "bwd_dkdv": 2.0 * F, "bwd_dq": 1.5 * F}
+    dom = max(kflops, key=lambda n: per[n])
+    kname = {"fwd": "fwd_kernel", "bwd_dkdv": "bwd_dkdv_kernel", "bwd_dq": "bwd_dq_kernel"}[dom]
+    achieved = kflops[dom] / (per[dom] * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": kname, "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic_for(kname),
+                "peak_source": f"{peaks_kind} {peak_key}",
+                "algorithmic_flops_per_launch": kflops[dom], "avg_launch_ms": round(per[dom], 4)}
+
+    decode = run_decode(args, torch, fa, _lib, workloads, dev, stream, world, peaks, peaks_kind)
+    e2e = run_e2e(args, torch, fa, w, q, k, v, do, dev, stream, world, F) if not args.no_e2e else None
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(q, k, v, do, w)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "GQA training step: fwd+bwd, B=1 Hq=32 Hkv=8 Nq=Nk=8192 d=128 causal bf16",
+                   "global_batch": B * world, "seq_len": N, "parallelism": f"replicas x{world} (weak)",
+                   "l2": "no flush: each step touches 320 MiB > 126 MB L2",
+                   "flops_convention": "fwd 4*B*Hq*N*N*d/2 (causal); bwd 2.5x fwd"},
+        "parts": {"fwd_ms": round(per["fwd"], 4), "fwd_tflops": round(fwd_tflops, 1),
+                  "fwd_frac_of_datasheet_2250": round(fwd_tflops / DENSE_BF16_DATASHEET_TFLOPS, 4),
+                  "fwd_frac_of_measured": round(fwd_tflops / peak, 4),
+                  "bwd_ms": round(bwd_ms, 4), "bwd_tflops": round(bwd_tflops, 1),
+                  "bwd_frac_of_datasheet_2250": round(bwd_tflops / DENSE_BF16_DATASHEET_TFLOPS, 4),
+                  "bwd_frac_of_measured": round(bwd_tflops / peak, 4),
+                  "per_kernel_ms": {kk: round(vv, 4) for kk, vv in per.items()}},
+        "decode": decode,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 4 * K,
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_decode(args, torch, fa, _lib, workloads, dev, stream, world, peaks, peaks_kind):
+    w = workloads.get(5)
+    q, kc, vc, sl = workloads.workload_inputs(w, device=dev)
+    sld = sl.to(dev)
+    B, Hq, Hkv, Nmax, d = w.B, w.Hq, w.Hkv, w.Nk, w.d
+    S = fa.fa_decode_num_splits(B, Hkv, Nmax, d, 0)
+    ws = torch.empty(fa.fa_decode_workspace_bytes(B, Hq, S, d), device=dev, dtype=torch.uint8)
+    o = torch.empty(B, 1, Hq, d, device=dev, dtype=torch.bfloat16)
+    lse = torch.empty(B, Hq, 1, device=dev, dtype=torch.float32)
+    sh = stream.cuda_stream
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        _lib.fa_decode_splitkv(q.data_ptr(), kc.data_ptr(), vc.data_ptr(), sld.data_ptr(), B, Hq, Hkv, Nmax, d,
+                               w.scale, S, ws.data_ptr(), _lib.FA_BF16, sh)
+        if ev:
+            ev[1].record(stream)
+        _lib.fa_decode_combine(ws.data_ptr(), o.data_ptr(), lse.data_ptr(), sld.data_ptr(), B, Hq, S, d,
+                               _lib.FA_BF16, sh)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    barrier(torch, world)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(torch, world)
+    ms = max_over_ranks(torch, world, t0.elapsed_time(t1)) / K
+    if fa.device_status() != 0:
+        raise RuntimeError("kernel status word set during decode")
+    split_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in evs)
+    comb_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in evs)
+    kv_bytes = int(sl.to(torch.int64).sum()) * Hkv * d * 2 * 2
+    q_bytes = B * Hq * d * 2
+    part_bytes = B * Hq * S * (d + 1) * 4
+    split_bytes = kv_bytes + q_bytes + part_bytes
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    gbs_step = world * (kv_bytes + q_bytes + B * Hq * d * 2) / (ms * 1e-3) / 1e9
+    gbs_split = split_bytes / (split_ms * 1e-3) / 1e9
+    return {"workload": "split-KV decode: B=64 Hq=32 Hkv=8 Nq=1 Nk_max=32768 (b>=32 ragged U[1024,32768]) d=128 bf16",
+            "num_splits": S, "ms_per_step": round(ms, 4), "split_ms": round(split_ms, 4),
+            "combine_ms": round(comb_ms, 4), "kv_bytes": kv_bytes, "value": round(gbs_step, 1), "unit": "GB/s",
+            "frac_of_measured_hbm": round(gbs_step / hbm, 4), "frac_of_8000": round(gbs_step / 8000.0, 4),
+            "roofline": {"bound": "hbm", "kernel": "decode_split_kernel", "achieved": round(gbs_split, 1),
+                         "peak": hbm, "unit": "GB/s", "frac": round(gbs_split / hbm, 4),
+                         "traffic": traffic_for("decode_split_kernel"), "peak_source": f"{peaks_kind} hbm_gbs",
+                         "algorithmic_bytes_per_launch": split_bytes},
+            "gpu_launches": 2 * K}
+
+
+def run_e2e(args, torch, fa, w, q, k, v, do, dev, stream, world, F):
+    """Same step through the public Python API with host buffers: pinned H2D of
+    q, k, v, dO, forward, backward, D2H of dQ, dK, dV, all inside the timed region."""
+    hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+    oq, ok_, ov = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (q, k, v))
+    dq_, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    qd, kd, vd, dod = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(do)
+    ws = torch.empty(fa.fa_bwd_workspace_bytes(w.B, w.Hq, w.Nq), device=dev, dtype=torch.uint8)
+
+    def step():
+        qd.copy_(hq, non_blocking=True)
+        kd.copy_(hk, non_blocking=True)
+        vd.copy_(hv, non_blocking=True)
+        dod.copy_(hdo, non_blocking=True)
+        o, lse = fa.attention_fwd(qd, kd, vd, causal=True)
+        fa.attention_bwd(qd, kd, vd, o, dod, lse, causal=True, workspace=ws, dq=dq_, dk=dk_, dv=dv_)
+        oq.copy_(dq_, non_blocking=True)
+        ok_.copy_(dk_, non_blocking=True)
+        ov.copy_(dv_, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(torch, world)
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(K):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(torch, world)
+    ms = max_over_ranks(torch, world, t0.elapsed_time(t1)) / K
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v, do))
+    d2h = sum(t.numel() * t.element_size() for t in (dq_, dk_, dv_))
+    return {"value": round(world * 3.5 * F / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def cpu_baseline(q, k, v, do, w):
+    """The fp64 oracle as it stands, on the host cores, on a bounded sample of the
+    same workload: KV group 0 (4 query heads) of the GQA training step, fwd + bwd."""
+    import numpy as np
+
+    import oracle
+    G = w.Hq // w.Hkv
+    qs = q[:, :, :G].float().cpu().numpy().astype(np.float64)
+    ks = k[:, :, :1].float().cpu().numpy().astype(np.float64)
+    vs = v[:, :, :1].float().cpu().numpy().astype(np.float64)
+    dos = do[:, :, :G].float().cpu().numpy().astype(np.float64)
+    threads = _blas_threads()
+    t = time.perf_counter()
+    oracle.attention_fwd(qs, ks, vs, True, w.scale)
+    oracle.attention_bwd(qs, ks, vs, dos, True, w.scale)
+    dt = time.perf_counter() - t
+    flops = 3.5 * attn_flops(1, G, w.Nq, w.Nk, w.d, True)
+    return {"value": round(flops / dt / 1e12, 5), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"KV group 0 ({G} query heads) of the GQA training step, fwd+bwd, {dt:.1f} s",
+            "seconds": round(dt, 2)}
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:  # noqa: BLE001
+        pass
+    return os.cpu_count()
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the fp64 oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    import oracle
+    import workloads
+    w = workloads.get(3)
+    q, k, v, do = workloads.workload_inputs(w)
+    # one query head and its KV head of the GQA training step, fwd + bwd, per step
+    qs, ks, vs, dos = (t[:, :, :1].float().numpy().astype(np.float64) for t in (q, k, v, do))
+    del torch
+
+    def step():
+        oracle.attention_fwd(qs, ks, vs, True, w.scale)
+        oracle.attention_bwd(qs, ks, vs, dos, True, w.scale)
+
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t) / args.steps
+    flops = 3.5 * attn_flops(1, 1, w.Nq, w.Nk, w.d, True)
+    val = flops / dt / 1e12
+    threads = _blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(val, 5), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "GQA training step: fwd+bwd, B=1 Hq=32 Hkv=8 Nq=Nk=8192 d=128 causal bf16 inputs",
+                   "sample": "one query head with its KV head per step", "global_batch": 1, "seq_len": w.Nq,
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(val, 5), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": "one query head with its KV head of the GQA training step, fwd+bwd"},
+        "e2e": {"value": round(val, 5), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

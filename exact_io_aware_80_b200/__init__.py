@@ -1,0 +1,129 @@
+"""Exact IO-aware attention on one B200: PyTorch-facing wrappers of libfa.so.
+
+The wrappers only check tensor metadata, allocate outputs and workspaces with
+PyTorch, and pass raw device pointers plus the current CUDA stream to the C
+entry points of the same names (see ``_lib``).  Every step of the attention
+computation runs in the CUDA kernels of libfa.so; there is no CPU or PyTorch
+fallback, and calling any of these without the built library or without a
+CUDA device raises.
+
+Layout (BSHD): q, o [B, Nq, Hq, d]; k, v [B, Nk, Hkv, d]; lse [B, Hq, Nq] fp32.
+"""
+from __future__ import annotations
+
+import math
+
+from . import _lib
+from ._lib import (FAError, fa_bwd, fa_bwd_dkdv, fa_bwd_dq, fa_bwd_preprocess, fa_bwd_workspace_bytes, fa_decode_chunk, fa_decode_combine,  # noqa: F401
+                   fa_decode_num_splits, fa_decode_splitkv, fa_decode_workspace_bytes, fa_fwd,
+                   fa_get_device_status, fa_version)
+
+__all__ = [
+    "attention_fwd", "attention_bwd", "decode", "decode_splitkv", "decode_combine", "device_status",
+    "fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq", "fa_decode_splitkv", "fa_decode_combine", "fa_decode_num_splits",
+    "fa_decode_workspace_bytes", "fa_bwd_workspace_bytes", "fa_decode_chunk", "fa_get_device_status",
+    "FAError",
+]
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dt(t):
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return _lib.FA_BF16
+    if t.dtype == torch.float16:
+        return _lib.FA_FP16
+    raise TypeError(f"attention tensors must be fp16 or bf16, got {t.dtype}")
+
+
+def _dev(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("libfa.so takes CUDA tensors only (no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous (BSHD)")
+    return ts[0].device
+
+
+def _stream(device):
+    return _torch().cuda.current_stream(device).cuda_stream
+
+
+def attention_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None):
+    """O, LSE = softmax(scale q k^T + mask) v, via ``fa_fwd``."""
+    torch = _torch()
+    dev = _dev(q, k, v)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty(B, Hq, Nq, device=dev, dtype=torch.float32) if lse is None else lse
+    fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
+           causal, scale, _dt(q), _stream(dev))
+    return o, l
+
+
+def attention_bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, workspace=None,
+                  dq=None, dk=None, dv=None):
+    """dQ, dK, dV of sum(dO * O), P recomputed from ``lse``, via ``fa_bwd``."""
+    torch = _torch()
+    dev = _dev(q, k, v, o, do, lse)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(fa_bwd_workspace_bytes(B, Hq, Nq), device=dev, dtype=torch.uint8)
+    fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+           dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), B, Hq, Hkv, Nq, Nk, d, causal, scale, _dt(q),
+           _stream(dev))
+    return dq, dk, dv
+
+
+def decode_splitkv(q, k_cache, v_cache, seqlens_k, num_splits: int, scale: float | None = None, workspace=None):
+    """Per-split partials of one-token decode (``fa_decode_splitkv``); returns the workspace."""
+    torch = _torch()
+    dev = _dev(q, k_cache, v_cache, seqlens_k)
+    B, _, Hq, d = q.shape
+    _, Nk_max, Hkv, _ = k_cache.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if workspace is None:
+        workspace = torch.empty(fa_decode_workspace_bytes(B, Hq, num_splits, d), device=dev, dtype=torch.uint8)
+    fa_decode_splitkv(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens_k.data_ptr(), B, Hq, Hkv,
+                      Nk_max, d, scale, num_splits, workspace.data_ptr(), _dt(q), _stream(dev))
+    return workspace
+
+
+def decode_combine(workspace, seqlens_k, B, Hq, d, num_splits, dtype, out=None, lse=None):
+    """Log-sum-exp merge of the split partials (``fa_decode_combine``)."""
+    torch = _torch()
+    dev = _dev(workspace, seqlens_k)
+    o = torch.empty(B, 1, Hq, d, device=dev, dtype=dtype) if out is None else out
+    l = torch.empty(B, Hq, 1, device=dev, dtype=torch.float32) if lse is None else lse
+    dt = _lib.FA_BF16 if dtype == torch.bfloat16 else _lib.FA_FP16
+    fa_decode_combine(workspace.data_ptr(), o.data_ptr(), l.data_ptr(), seqlens_k.data_ptr(), B, Hq, num_splits, d,
+                      dt, _stream(dev))
+    return o, l
+
+
+def decode(q, k_cache, v_cache, seqlens_k, num_splits: int | None = None, scale: float | None = None,
+           workspace=None, out=None, lse=None):
+    """One-token split-KV decode: partial pass then combine."""
+    B, _, Hq, d = q.shape
+    _, Nk_max, Hkv, _ = k_cache.shape
+    if num_splits is None:
+        num_splits = fa_decode_num_splits(B, Hkv, Nk_max, d, 0)
+    ws = decode_splitkv(q, k_cache, v_cache, seqlens_k, num_splits, scale, workspace)
+    return decode_combine(ws, seqlens_k, B, Hq, d, num_splits, q.dtype, out, lse)
+
+
+def device_status(stream=None) -> int:
+    """Synchronise and return (then clear) the kernels' device status word."""
+    s = _stream(_torch().cuda.current_device()) if stream is None else stream
+    return fa_get_device_status(s)

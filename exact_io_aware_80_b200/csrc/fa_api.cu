@@ -1,0 +1,242 @@
+// fa_api.cu -- the C ABI of libfa.so (declared in include/fa.h): argument
+// validation, workspace sizing, the split heuristic and kernel dispatch.
+// Validation happens before anything is launched; the library allocates no
+// device memory.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "kernels.h"
+
+namespace {
+
+// Device status word written by kernels whose bounded waits run out.  Host
+// code reaches it only through the address that cudaGetSymbolAddress returns
+// for the current device.
+__device__ int g_fa_status = 0;
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {nullptr};
+std::mutex g_status_mu;
+
+int* status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fa_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+fa_status check_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, fa_dtype dt) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID;
+  if (causal && Nq > Nk) return FA_ERR_INVALID;
+  if (dt != FA_FP16 && dt != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hq > 65535) return FA_ERR_UNSUPPORTED;
+  // every element index must fit the kernels' 64-bit offsets and the grid
+  if ((long long)Nq > (1ll << 30) || (long long)Nk > (1ll << 30)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+fa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return 1; }
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FA_ERR_ALIGN: return "pointer not aligned";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_TIMEOUT: return "kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                 int Nk, int d, int causal, float scale, fa_dtype dt, fa_stream_t stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID;
+  fa_status st = check_shape(B, Hq, Hkv, Nq, Nk, d, causal, dt);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse)) return FA_ERR_ALIGN;
+  fa::AttnArgs a{q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal ? 1 : 0, scale, dt == FA_BF16 ? 1 : 0, status_ptr()};
+  if (!a.status) return FA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (fa::fwd_sm100_supported(a)) return from_cuda(fa::launch_fwd_sm100(a, s));
+  return from_cuda(fa::launch_fwd_mma(a, s));
+}
+
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq) {
+  if (B < 1 || Hq < 1 || Nq < 1) return 0;
+  return (size_t)B * Hq * Nq * sizeof(float);
+}
+
+// step bits for bwd_run
+enum { kPre = 1, kDkdv = 2, kDq = 4 };
+
+static fa_status bwd_run(int steps, const void* q, const void* k, const void* v, const void* o, const void* dout,
+                         const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv,
+                         int Nq, int Nk, int d, int causal, float scale, fa_dtype dt, fa_stream_t stream) {
+  const bool pre = steps & kPre, dkdv = steps & kDkdv, dqs = steps & kDq;
+  if (!workspace || !dout) return FA_ERR_INVALID;
+  if (pre && !o) return FA_ERR_INVALID;
+  if ((dkdv || dqs) && (!q || !k || !v || !lse)) return FA_ERR_INVALID;
+  if (dkdv && (!dk || !dv)) return FA_ERR_INVALID;
+  if (dqs && !dq) return FA_ERR_INVALID;
+  fa_status st = check_shape(B, Hq, Hkv, Nq, Nk, d, causal, dt);
+  if (st != FA_OK) return st;
+  const void* p16[] = {q, k, v, o, dout, dq, dk, dv, workspace};
+  for (const void* p : p16)
+    if (p && !aligned16(p)) return FA_ERR_ALIGN;
+  if (lse && !aligned4(lse)) return FA_ERR_ALIGN;
+  fa::BwdArgs a{q, k, v, o, dout, lse, dq, dk, dv, static_cast<float*>(workspace), B, Hq, Hkv, Nq, Nk, d,
+                causal ? 1 : 0, scale, dt == FA_BF16 ? 1 : 0, status_ptr()};
+  if (!a.status) return FA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (pre) e = fa::launch_bwd_preprocess(a, s);
+  if (e == cudaSuccess && dkdv) e = fa::launch_bwd_dkdv(a, s);
+  if (e == cudaSuccess && dqs) e = fa::launch_bwd_dq(a, s);
+  return from_cuda(e);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                 void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                 int causal, float scale, fa_dtype dt, fa_stream_t stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID;
+  return bwd_run(kPre | kDkdv | kDq, q, k, v, o, dout, lse, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, causal,
+                 scale, dt, stream);
+}
+
+fa_status fa_bwd_preprocess(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                            const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv,
+                            int Nq, int Nk, int d, int causal, float scale, fa_dtype dt, fa_stream_t stream) {
+  return bwd_run(kPre, q, k, v, o, dout, lse, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, causal, scale, dt,
+                 stream);
+}
+
+fa_status fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                      void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                      int causal, float scale, fa_dtype dt, fa_stream_t stream) {
+  return bwd_run(kDkdv, q, k, v, o, dout, lse, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, causal, scale, dt,
+                 stream);
+}
+
+fa_status fa_bwd_dq(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                    void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                    int causal, float scale, fa_dtype dt, fa_stream_t stream) {
+  return bwd_run(kDq, q, k, v, o, dout, lse, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, causal, scale, dt,
+                 stream);
+}
+
+int fa_decode_chunk(int Nk_max, int num_splits) {
+  if (Nk_max < 1 || num_splits < 1) return 64;
+  int c = (Nk_max + num_splits - 1) / num_splits;
+  return ((c + 63) / 64) * 64;
+}
+
+int fa_decode_num_splits(int B, int Hkv, int Nk_max, int d, int num_sms) {
+  (void)d;
+  if (B < 1 || Hkv < 1 || Nk_max < 1) return 1;
+  if (num_sms <= 0) {
+    int dev = 0;
+    num_sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+      int n = 0;
+      if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) num_sms = n;
+    }
+  }
+  const long long units = (long long)B * Hkv;
+  const int max_splits = (Nk_max + 63) / 64;
+  // Aim at >= 8 waves of (b, h_kv, split) units so that the ragged lengths of
+  // a batch even out across SMs, with splits of at least 256 keys.
+  long long want = (8ll * num_sms + units - 1) / units;
+  int splits = (int)(want < 1 ? 1 : want);
+  const int min_keys = 256;
+  const int cap = (Nk_max + min_keys - 1) / min_keys;
+  if (splits > cap) splits = cap;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  // drop trailing splits that the 64-key rounding of the chunk left empty
+  const int chunk = fa_decode_chunk(Nk_max, splits);
+  return (Nk_max + chunk - 1) / chunk;
+}
+
+size_t fa_decode_workspace_bytes(int B, int Hq, int num_splits, int d) {
+  if (B < 1 || Hq < 1 || num_splits < 1 || d < 1) return 0;
+  const size_t o = (size_t)B * Hq * num_splits * d * sizeof(float);
+  const size_t l = (size_t)B * Hq * num_splits * sizeof(float);
+  return o + ((l + 255) / 256) * 256;
+}
+
+static fa_status decode_check(int B, int Hq, int Hkv, int Nk_max, int d, int num_splits, fa_dtype dt) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nk_max < 1 || num_splits < 1) return FA_ERR_INVALID;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID;
+  if (dt != FA_FP16 && dt != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 16) return FA_ERR_UNSUPPORTED;  // one CTA holds a GQA group of at most 16 query heads
+  if (B > 65535 || Hkv > 65535 || Hq > 65535 || num_splits > 65535) return FA_ERR_UNSUPPORTED;
+  if (num_splits > (Nk_max + 63) / 64) return FA_ERR_INVALID;
+  return FA_OK;
+}
+
+fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k, int B,
+                            int Hq, int Hkv, int Nk_max, int d, float scale, int num_splits, void* workspace,
+                            fa_dtype dt, fa_stream_t stream) {
+  if (!q || !k_cache || !v_cache || !seqlens_k || !workspace) return FA_ERR_INVALID;
+  fa_status st = decode_check(B, Hq, Hkv, Nk_max, d, num_splits, dt);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(workspace) || !aligned4(seqlens_k))
+    return FA_ERR_ALIGN;
+  float* o_part = static_cast<float*>(workspace);
+  float* lse_part = o_part + (size_t)B * Hq * num_splits * d;
+  fa::DecodeArgs a{q,     k_cache, v_cache,    seqlens_k, o_part, lse_part, B, Hq, Hkv, Nk_max, d, num_splits,
+                   fa_decode_chunk(Nk_max, num_splits), scale, dt == FA_BF16 ? 1 : 0, status_ptr()};
+  if (!a.status) return FA_ERR_CUDA;
+  return from_cuda(fa::launch_decode_split(a, static_cast<cudaStream_t>(stream)));
+}
+
+fa_status fa_decode_combine(const void* workspace, void* o, float* lse, const int* seqlens_k, int B, int Hq,
+                            int num_splits, int d, fa_dtype dt, fa_stream_t stream) {
+  if (!workspace || !o || !lse || !seqlens_k) return FA_ERR_INVALID;
+  if (B < 1 || Hq < 1 || num_splits < 1) return FA_ERR_INVALID;
+  if (dt != FA_FP16 && dt != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hq > 65535) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(workspace) || !aligned16(o) || !aligned4(lse) || !aligned4(seqlens_k)) return FA_ERR_ALIGN;
+  const float* o_part = static_cast<const float*>(workspace);
+  const float* lse_part = o_part + (size_t)B * Hq * num_splits * d;
+  fa::CombineArgs a{o_part, lse_part, seqlens_k, o, lse, B, Hq, d, num_splits, dt == FA_BF16 ? 1 : 0};
+  return from_cuda(fa::launch_decode_combine(a, static_cast<cudaStream_t>(stream)));
+}
+
+fa_status fa_get_device_status(fa_stream_t stream) {
+  int* p = status_ptr();
+  if (!p) return FA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return static_cast<fa_status>(v);
+}
+
+}  // extern "C"

@@ -1,0 +1,78 @@
+// kernels.h -- host-side launchers of the attention kernels (internal to libfa.so).
+// Arguments are validated by the C ABI in fa_api.cu before any launcher runs.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa {
+
+struct AttnArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  int B, Hq, Hkv, Nq, Nk, d;
+  int causal;
+  float scale;
+  int bf16;  // 1: bf16, 0: fp16
+  int* status;
+};
+
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* dout;
+  const float* lse;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* dvec;  // D [B,Hq,Nq] fp32 workspace
+  int B, Hq, Hkv, Nq, Nk, d;
+  int causal;
+  float scale;
+  int bf16;
+  int* status;
+};
+
+struct DecodeArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const int* seqlens;
+  float* o_part;    // [B,Hq,S,d]
+  float* lse_part;  // [B,Hq,S]
+  int B, Hq, Hkv, Nk_max, d;
+  int num_splits, chunk;
+  float scale;
+  int bf16;
+  int* status;
+};
+
+struct CombineArgs {
+  const float* o_part;
+  const float* lse_part;
+  const int* seqlens;
+  void* o;
+  float* lse;
+  int B, Hq, d, num_splits;
+  int bf16;
+};
+
+// Forward on legacy warp-level MMA (mma.sync m16n8k16), FA-2 style work split.
+cudaError_t launch_fwd_mma(const AttnArgs& a, cudaStream_t s);
+// Forward on tcgen05 / TMEM / TMA (warp-specialised), d = 128 and 64.
+cudaError_t launch_fwd_sm100(const AttnArgs& a, cudaStream_t s);
+bool fwd_sm100_supported(const AttnArgs& a);
+
+cudaError_t launch_bwd_preprocess(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_dkdv(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_dq(const BwdArgs& a, cudaStream_t s);
+
+cudaError_t launch_decode_split(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode_combine(const CombineArgs& a, cudaStream_t s);
+
+}  // namespace fa

@@ -89,6 +89,30 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  fa_dtype dt, fa_stream_t stream);
 
 /*
+ * The three launches fa_bwd makes, callable one by one (same arguments, same
+ * validation), so that a caller can time or schedule them separately:
+ *   fa_bwd_preprocess: workspace D[b,h,i] = sum_c dout[b,i,h,c] * o[b,i,h,c] (fp32);
+ *   fa_bwd_dkdv: dk, dv from q, k, v, dout, lse and D (one CTA per 64-key tile
+ *     of a KV head, looping over its group's query heads and query tiles);
+ *   fa_bwd_dq: dq from q, k, v, dout, lse and D (one CTA per 64-row query tile).
+ * fa_bwd_dkdv and fa_bwd_dq read the D that fa_bwd_preprocess wrote, so on one
+ * stream the preprocess call must come first.  Arguments a step does not read
+ * may be NULL (preprocess: q, k, v, lse, dq, dk, dv; dkdv: o, dq; dq: o, dk, dv).
+ */
+fa_status fa_bwd_preprocess(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                            const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                            int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                            fa_dtype dt, fa_stream_t stream);
+fa_status fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                      const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                      int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                      fa_dtype dt, fa_stream_t stream);
+fa_status fa_bwd_dq(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                    const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                    int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                    fa_dtype dt, fa_stream_t stream);
+
+/*
  * Suggested number of key splits for fa_decode_splitkv: enough (b, h_kv, split)
  * units to fill `num_sms` SMs several times over (num_sms <= 0: query the
  * current device).  Always >= 1 and <= ceil(Nk_max / 64).

@@ -61,6 +61,8 @@ __all__ = [
     "attention_fwd_rows",
     "attention_fwd_online",
     "attention_bwd",
+    "attention_bwd_dq_rows",
+    "attention_bwd_kv_rows",
     "bwd_preprocess",
     "decode",
     "decode_splitkv",
@@ -258,6 +260,56 @@ def attention_bwd(q, k, v, do, causal: bool, scale: float, kv_heads=None):
         dk[b, :, hk, :] = dK
         dv[b, :, hk, :] = dV
     return dq, dk, dv
+
+
+def attention_bwd_dq_rows(q, k, v, do, causal: bool, scale: float, b: int, h: int, rows):
+    """dQ for selected query rows of one (b, h_q), row by row.
+
+    Every quantity dQ_i needs is a function of row i alone: its scores S_i,
+    its softmax P_i, O_i = P_i V, D_i = dO_i . O_i, dP_i = dO_i V^T,
+    dS_i = P_i (dP_i - D_i) and dQ_i = scale dS_i K.  Returns [len(rows), d].
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, Nq, Nk, Hq, Hkv, d = _check_shapes(q, k, v)
+    hk = h // (Hq // Hkv)
+    rows = np.asarray(rows, dtype=np.int64)
+    K, V = k[b, :, hk, :], v[b, :, hk, :]
+    P, _ = softmax_rows(scores(q[b, rows, h, :], K, scale, visible_mask(Nq, Nk, causal)[rows]))
+    dO = do[b, rows, h, :]
+    O = P @ V
+    D = np.sum(dO * O, axis=1, keepdims=True)
+    dS = P * (dO @ V.T - D)
+    return scale * (dS @ K)
+
+
+def attention_bwd_kv_rows(q, k, v, do, causal: bool, scale: float, b: int, hk: int, keys, row_chunk: int = 1024):
+    """dK and dV for selected key rows j of one (b, h_kv).
+
+    dK_j = scale sum_{h in group} sum_i dS_ij Q_i and dV_j = sum_h sum_i P_ij dO_i
+    need column j of P and dS for every query row i; each row's softmax still
+    needs its whole score row, so the query rows are visited in chunks of
+    ``row_chunk`` (to bound memory), each chunk evaluated exactly as in
+    ``attention_bwd``.  Returns ([len(keys), d], [len(keys), d]).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, Nq, Nk, Hq, Hkv, d = _check_shapes(q, k, v)
+    G = Hq // Hkv
+    keys = np.asarray(keys, dtype=np.int64)
+    K, V = k[b, :, hk, :], v[b, :, hk, :]
+    mask = visible_mask(Nq, Nk, causal)
+    dK = np.zeros((len(keys), d))
+    dV = np.zeros((len(keys), d))
+    for h in range(hk * G, (hk + 1) * G):
+        for i0 in range(0, Nq, row_chunk):
+            rows = slice(i0, min(i0 + row_chunk, Nq))
+            Q, dO = q[b, rows, h, :], do[b, rows, h, :]
+            P, _ = softmax_rows(scores(Q, K, scale, mask[rows]))
+            D = np.sum(dO * (P @ V), axis=1, keepdims=True)
+            Pj = P[:, keys]
+            dSj = Pj * (dO @ V[keys].T - D)
+            dV += Pj.T @ dO
+            dK += scale * (dSj.T @ Q)
+    return dK, dV
 
 
 def decode(q, k_cache, v_cache, seqlens_k, scale: float):

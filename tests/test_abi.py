@@ -1,0 +1,128 @@
+"""Host-side checks of libfa.so that need no GPU: the library loads, exports
+every entry point include/fa.h declares, and validation rejects bad
+arguments before anything is launched (so fake pointers are never touched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_io_aware_80_b200 import build, _lib
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(fa_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("fa_fwd", "fa_bwd", "fa_decode_splitkv", "fa_decode_combine", "fa_get_device_status"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from exact_io_aware_80_b200 import _lib
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+        assert n in _lib.SIGNATURES, f"binding lacks {n}"
+
+
+def test_status_strings_and_version(lib):
+    from exact_io_aware_80_b200 import _lib
+    assert _lib.fa_version() >= 1
+    for code in (0, -1, -2, -3, -4, -5):
+        assert _lib.status_string(code)
+
+
+def test_workspace_sizes(lib):
+    from exact_io_aware_80_b200 import _lib
+    assert _lib.fa_bwd_workspace_bytes(1, 32, 8192) == 32 * 8192 * 4
+    ws = _lib.fa_decode_workspace_bytes(64, 32, 16, 128)
+    assert ws >= 64 * 32 * 16 * 128 * 4 + 64 * 32 * 16 * 4
+    assert ws % 16 == 0
+
+
+def test_decode_chunk_and_splits(lib):
+    from exact_io_aware_80_b200 import _lib
+    assert _lib.fa_decode_chunk(32768, 16) == 2048
+    assert _lib.fa_decode_chunk(1000, 3) == 384
+    for B, Hkv, N in ((64, 8, 32768), (1, 1, 1), (1, 8, 100000), (256, 8, 512)):
+        s = _lib.fa_decode_num_splits(B, Hkv, N, 128, 148)
+        assert 1 <= s <= -(-N // 64)
+        # the last split must not start past the cache
+        assert (s - 1) * _lib.fa_decode_chunk(N, s) < N or s == 1
+
+
+FAKE = 0x10000  # never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), -1),
+    (dict(Hq=6, Hkv=4), -1),
+    (dict(causal=1, Nq=10, Nk=5), -1),
+    (dict(d=96), -2),
+    (dict(d=256), -2),
+    (dict(dt=7), -2),
+    (dict(B=0), -1),
+    (dict(q=FAKE + 8), -3),
+])
+def test_fwd_rejects_bad_arguments(lib, kw, code):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=4, Hkv=2, Nq=8, Nk=8, d=128, causal=0,
+             scale=0.1, dt=1, stream=None)
+    a.update(kw)
+    rc = lib.fa_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Nq"], a["Nk"],
+                    a["d"], a["causal"], a["scale"], a["dt"], a["stream"])
+    assert rc == code
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    # only invalid argument lists are passed: a valid one would launch on fake pointers
+    args = [FAKE] * 10 + [1, 4, 2, 8, 8, 128, 0, 0.1, 1, None]
+    bad = list(args)
+    bad[9] = None  # workspace
+    assert lib.fa_bwd(*bad) == -1
+    bad = list(args)
+    bad[15] = 80  # d
+    assert lib.fa_bwd(*bad) == -2
+    bad = list(args)
+    bad[3] = FAKE + 4  # o misaligned
+    assert lib.fa_bwd(*bad) == -3
+
+
+def test_decode_rejects_bad_arguments(lib):
+    # q, kc, vc, seqlens, B, Hq, Hkv, Nk_max, d, scale, splits, ws, dt, stream
+    base = [FAKE, FAKE, FAKE, FAKE, 2, 32, 8, 1024, 128, 0.1, 4, FAKE, 1, None]
+    bad = list(base)
+    bad[5] = 33  # Hq % Hkv
+    assert lib.fa_decode_splitkv(*bad) == -1
+    bad = list(base)
+    bad[5], bad[6] = 64, 2  # group of 32 > 16
+    assert lib.fa_decode_splitkv(*bad) == -2
+    bad = list(base)
+    bad[10] = 17  # more splits than 64-key tiles
+    assert lib.fa_decode_splitkv(*bad) == -1
+    bad = list(base)
+    bad[3] = FAKE + 2  # seqlens misaligned
+    assert lib.fa_decode_splitkv(*bad) == -3
+    assert lib.fa_decode_combine(FAKE, FAKE, FAKE, FAKE, 2, 32, 0, 128, 1, None) == -1
+    assert lib.fa_decode_combine(FAKE, FAKE, FAKE, FAKE, 2, 32, 4, 72, 1, None) == -2
+
+
+def test_binding_without_gpu_fails_loudly():
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    import exact_io_aware_80_b200 as fa
+    q = torch.zeros(1, 8, 2, 64, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        fa.attention_fwd(q, q, q)

@@ -249,6 +249,20 @@ def test_preprocess_equals_rowsum_p_dp():
         np.testing.assert_allclose(D[0, h], (P * dP).sum(axis=1), atol=1e-12)
 
 
+def test_backward_sampled_rows_match_full():
+    q, k, v = tiny(B=2, Hq=4, Hkv=2, Nq=7, Nk=9, d=3)
+    do = rnd(*q.shape)
+    for causal in (False, True):
+        dq, dk, dv = oracle.attention_bwd(q, k, v, do, causal, 0.5)
+        rows = [0, 3, 6]
+        np.testing.assert_allclose(oracle.attention_bwd_dq_rows(q, k, v, do, causal, 0.5, 1, 2, rows),
+                                   dq[1, rows, 2], atol=1e-13)
+        keys = [0, 4, 8]
+        dk_s, dv_s = oracle.attention_bwd_kv_rows(q, k, v, do, causal, 0.5, 1, 1, keys, row_chunk=3)
+        np.testing.assert_allclose(dk_s, dk[1, keys, 1], atol=1e-13)
+        np.testing.assert_allclose(dv_s, dv[1, keys, 1], atol=1e-13)
+
+
 def test_backward_head_subset_matches_full():
     q, k, v = tiny(B=2, Hq=4, Hkv=2, Nq=5, Nk=5, d=3)
     do = rnd(*q.shape)
