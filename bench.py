@@ -182,6 +182,9 @@ def run_ours(args):
     peaks, peaks_kind = load_peaks()
 
     w = workloads.get(3)
+    if args.seq:
+        import dataclasses
+        w = dataclasses.replace(w, Nq=args.seq, Nk=args.seq)
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.Nq, w.d
     q, k, v, do = workloads.workload_inputs(w, device=dev)
     o = torch.empty_like(q)
@@ -259,20 +262,22 @@ def run_ours(args):
                 "peak_source": f"{peaks_kind} {peak_key}",
                 "algorithmic_flops_per_launch": kflops[dom], "avg_launch_ms": round(per[dom], 4)}
 
-    decode = run_decode(args, torch, fa, _lib, workloads, dev, stream, world, peaks, peaks_kind)
+    decode = None if args.no_decode else run_decode(args, torch, fa, _lib, workloads, dev, stream, world, peaks,
+                                                    peaks_kind)
     e2e = run_e2e(args, torch, fa, w, q, k, v, do, dev, stream, world, F) if not args.no_e2e else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(q, k, v, do, w)
 
+    touched = sum(t.numel() * t.element_size() for t in (q, k, v, o, do, dq, dk, dv, lse, ws))
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "GQA training step: fwd+bwd, B=1 Hq=32 Hkv=8 Nq=Nk=8192 d=128 causal bf16",
+        "config": {"workload": f"GQA training step: fwd+bwd, B=1 Hq=32 Hkv=8 Nq=Nk={N} d=128 causal bf16",
                    "global_batch": B * world, "seq_len": N, "parallelism": f"replicas x{world} (weak)",
-                   "l2": "no flush: each step touches 320 MiB > 126 MB L2",
+                   "l2": f"no flush: each step touches {touched / 2**20:.0f} MiB (> 126 MB L2 at N=8192)",
                    "flops_convention": "fwd 4*B*Hq*N*N*d/2 (causal); bwd 2.5x fwd"},
         "parts": {"fwd_ms": round(per["fwd"], 4), "fwd_tflops": round(fwd_tflops, 1),
                   "fwd_frac_of_datasheet_2250": round(fwd_tflops / DENSE_BF16_DATASHEET_TFLOPS, 4),
@@ -297,6 +302,9 @@ def run_ours(args):
 
 def run_decode(args, torch, fa, _lib, workloads, dev, stream, world, peaks, peaks_kind):
     w = workloads.get(5)
+    if args.decode_b:
+        import dataclasses
+        w = dataclasses.replace(w, B=args.decode_b)
     q, kc, vc, sl = workloads.workload_inputs(w, device=dev)
     sld = sl.to(dev)
     B, Hq, Hkv, Nmax, d = w.B, w.Hq, w.Hkv, w.Nk, w.d
@@ -343,7 +351,8 @@ def run_decode(args, torch, fa, _lib, workloads, dev, stream, world, peaks, peak
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     gbs_step = world * (kv_bytes + q_bytes + B * Hq * d * 2) / (ms * 1e-3) / 1e9
     gbs_split = split_bytes / (split_ms * 1e-3) / 1e9
-    return {"workload": "split-KV decode: B=64 Hq=32 Hkv=8 Nq=1 Nk_max=32768 (b>=32 ragged U[1024,32768]) d=128 bf16",
+    return {"workload": f"split-KV decode: B={B} Hq=32 Hkv=8 Nq=1 Nk_max=32768 (b>={B // 2} ragged U[1024,32768]) "
+                        "d=128 bf16",
             "num_splits": S, "ms_per_step": round(ms, 4), "split_ms": round(split_ms, 4),
             "combine_ms": round(comb_ms, 4), "kv_bytes": kv_bytes, "value": round(gbs_step, 1), "unit": "GB/s",
             "frac_of_measured_hbm": round(gbs_step / hbm, 4), "frac_of_8000": round(gbs_step / 8000.0, 4),
@@ -480,6 +489,11 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode section (profiling runs)")
+    ap.add_argument("--decode-b", type=int, default=0,
+                    help="override B of the decode workload (profiling runs on a smaller case)")
+    ap.add_argument("--seq", type=int, default=0,
+                    help="override N of the training-step workload (profiling runs on a smaller case)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -119,13 +119,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(DecodeArgs p)
     float rs[2] = {0.f, 0.f};
 #pragma unroll
     for (int nb = 0; nb < 2; ++nb) {
-      const uint32_t plo = Elem<T>::pack(ex2(fmaf(sc[nb][0], c, -mu[0])), ex2(fmaf(sc[nb][1], c, -mu[0])));
-      const uint32_t phi = Elem<T>::pack(ex2(fmaf(sc[nb][2], c, -mu[1])), ex2(fmaf(sc[nb][3], c, -mu[1])));
-      const float2 fl = Elem<T>::unpack(plo), fh = Elem<T>::unpack(phi);
-      rs[0] += fl.x + fl.y;
-      rs[1] += fh.x + fh.y;
-      pa[nb * 2 + 0] = plo;
-      pa[nb * 2 + 1] = phi;
+      const float p0 = ex2(fmaf(sc[nb][0], c, -mu[0])), p1 = ex2(fmaf(sc[nb][1], c, -mu[0]));
+      const float p2 = ex2(fmaf(sc[nb][2], c, -mu[1])), p3 = ex2(fmaf(sc[nb][3], c, -mu[1]));
+      rs[0] += p0 + p1;
+      rs[1] += p2 + p3;
+      pa[nb * 2 + 0] = Elem<T>::pack(p0, p1);
+      pa[nb * 2 + 1] = Elem<T>::pack(p2, p3);
     }
     l_run[0] = l_run[0] * corr[0] + rs[0];
     l_run[1] = l_run[1] * corr[1] + rs[1];

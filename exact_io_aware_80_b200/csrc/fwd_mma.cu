@@ -7,8 +7,9 @@
 //   t = s * scale * log2(e),  m' = max(m, rowmax t),  p = 2^(t - m'),
 //   l = 2^(m - m') l + rowsum p,  O = 2^(m - m') O + P V,
 // and at the end O /= l, LSE = ln2 * (m + log2 l).  P is rounded to the input
-// dtype for the PV product and l is summed from the same rounded values, so
-// the weights applied to V sum to one.
+// dtype for the PV product; l is summed from the unrounded fp32 values, so
+// the LSE carries only fp32 rounding (the 16-bit rounding of P would move it
+// by up to 2^-9 relative).
 //
 // This is the compact, portable forward (any Nq, Nk, d in {64, 128}); the
 // tcgen05 kernel in fwd_sm100.cu is the fast path for sm_100a.
@@ -124,13 +125,12 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_mma_kernel(AttnArgs p) {
     float rs[2] = {0.f, 0.f};
 #pragma unroll
     for (int nb = 0; nb < kBN / 8; ++nb) {
-      const uint32_t lo = Elem<T>::pack(ex2(fmaf(s[nb][0], c, -mu[0])), ex2(fmaf(s[nb][1], c, -mu[0])));
-      const uint32_t hi = Elem<T>::pack(ex2(fmaf(s[nb][2], c, -mu[1])), ex2(fmaf(s[nb][3], c, -mu[1])));
-      const float2 fl = Elem<T>::unpack(lo), fh = Elem<T>::unpack(hi);
-      rs[0] += fl.x + fl.y;
-      rs[1] += fh.x + fh.y;
-      pa[nb >> 1][(nb & 1) * 2 + 0] = lo;
-      pa[nb >> 1][(nb & 1) * 2 + 1] = hi;
+      const float p0 = ex2(fmaf(s[nb][0], c, -mu[0])), p1 = ex2(fmaf(s[nb][1], c, -mu[0]));
+      const float p2 = ex2(fmaf(s[nb][2], c, -mu[1])), p3 = ex2(fmaf(s[nb][3], c, -mu[1]));
+      rs[0] += p0 + p1;
+      rs[1] += p2 + p3;
+      pa[nb >> 1][(nb & 1) * 2 + 0] = Elem<T>::pack(p0, p1);
+      pa[nb >> 1][(nb & 1) * 2 + 1] = Elem<T>::pack(p2, p3);
     }
     l_run[0] = l_run[0] * corr[0] + rs[0];
     l_run[1] = l_run[1] * corr[1] + rs[1];
