@@ -77,8 +77,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   fa::AttnArgs a{q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal ? 1 : 0, scale, dt == FA_BF16 ? 1 : 0, status_ptr()};
   if (!a.status) return FA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (fa::fwd_sm100_supported(a)) return from_cuda(fa::launch_fwd_sm100(a, s));
-  return from_cuda(fa::launch_fwd_mma(a, s));
+  if (!fa::fwd_sm100_supported(a)) return FA_ERR_CUDA;  // the driver lacks the tensor-map encoder
+  return from_cuda(fa::launch_fwd_sm100(a, s));
 }
 
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq) {

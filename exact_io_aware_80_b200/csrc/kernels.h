@@ -62,8 +62,6 @@ struct CombineArgs {
   int bf16;
 };
 
-// Forward on legacy warp-level MMA (mma.sync m16n8k16), FA-2 style work split.
-cudaError_t launch_fwd_mma(const AttnArgs& a, cudaStream_t s);
 // Forward on tcgen05 / TMEM / TMA (warp-specialised), d = 128 and 64.
 cudaError_t launch_fwd_sm100(const AttnArgs& a, cudaStream_t s);
 bool fwd_sm100_supported(const AttnArgs& a);
