@@ -149,6 +149,39 @@ fa_status fa_decode_combine(const void* workspace, void* o, float* lse, const in
 int fa_decode_chunk(int Nk_max, int num_splits);
 
 /*
+ * Split-KV decode that allocates nothing and takes no workspace.  The pages
+ * have no counterpart: this exists for callers that cannot allocate device
+ * memory -- a serving runtime that plans all device memory up front and
+ * forbids allocation on the request path, code running inside another
+ * library's allocator callback (allocating would re-enter it), or a
+ * latency-bound caller that cannot pay for a fresh allocation.
+ *
+ * Same inputs, outputs and result as fa_decode_splitkv followed by
+ * fa_decode_combine (q [B,1,Hq,d], caches [B,Nk_max,Hkv,d], seqlens_k device
+ * int32 [B], o [B,1,Hq,d], lse [B,Hq,1] fp32), computed by the same kernels;
+ * the split partials live in a static device array of
+ * FA_DECODE_NOALLOC_SCRATCH_BYTES bytes inside libfa.so, which every GPU that
+ * loads the library holds until the process exits.
+ *  - Size limit: the partials take B*Hq*S*d*4 bytes, rounded up to 256, plus
+ *    B*Hq*S*4 bytes for S splits; a request beyond the array returns
+ *    FA_ERR_UNSUPPORTED before anything is launched.  num_splits <= 0 takes the
+ *    fa_decode_num_splits suggestion, reduced until the partials fit.
+ *  - First call on a device: looks up the array's device address with
+ *    cudaGetSymbolAddress (with that device current) and keeps it; make that
+ *    first call before any stream capture on the device.
+ *  - Every call on a device shares the one array, which keeps the last call's
+ *    contents.  Calls whose kernels overlap on the GPU (two streams, or two host
+ *    threads without ordering) race on it; issue them on one stream.  Nothing
+ *    needs to start at zero: every partial the combine reads is written first
+ *    by the same call.
+ * Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define FA_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+fa_status fa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k,
+                            void* o, float* lse, int B, int Hq, int Hkv, int Nk_max, int d, float scale,
+                            int num_splits, fa_dtype dt, fa_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word that the
  * kernels set when a bounded wait runs out (FA_ERR_TIMEOUT) or a device-side
  * check fails.  Returns FA_OK when no kernel reported an error.
