@@ -255,7 +255,7 @@ def run_ours(args):
     # FLOPs each kernel must execute: fwd 2 GEMMs (F), dK/dV 4 GEMMs (2F), dQ 3 GEMMs (1.5F)
     kflops = {"fwd": F, "bwd_dkdv": 2.0 * F, "bwd_dq": 1.5 * F}
     dom = max(kflops, key=lambda n: per[n])
-    kname = {"fwd": "fwd_kernel", "bwd_dkdv": "bwd_dkdv_kernel", "bwd_dq": "bwd_dq_kernel"}[dom]
+    kname = {"fwd": "fwd_sm100_kernel", "bwd_dkdv": "bwd_dkdv_sm100_kernel", "bwd_dq": "bwd_dq_sm100_kernel"}[dom]
     achieved = kflops[dom] / (per[dom] * 1e-3) / 1e12
     roofline = {"bound": "tensor", "kernel": kname, "achieved": round(achieved, 1), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic_for(kname),

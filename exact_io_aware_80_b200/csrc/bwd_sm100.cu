@@ -1,0 +1,644 @@
+// bwd_sm100.cu -- attention backward on the sm_100a tensor-core path (TMA,
+// tcgen05 MMAs with accumulators in tensor memory, warp-specialised roles).
+//
+// The gradients are the chain rule of the definition, with P recomputed from
+// the stored log-sum-exp ("FlashAttention 심층 분석", section 4: keep only the
+// softmax statistics, rebuild P on chip):
+//   P = exp(scale q.k - LSE),  dP = dO V^T,  dS = P * (dP - D),  D = rowsum(dO * O)
+//   dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
+// Two kernels, no atomics (bitwise-reproducible results):
+//
+// dK/dV: one CTA per (128-key tile, KV head, batch).  K and V stay in shared
+//   memory; Q and dO tiles of the group's query heads stream through a
+//   two-stage TMA ring.  TMEM holds S^T (keys x queries, later P^T as 16-bit
+//   pairs), dP^T (later dS^T), and the dV and dK accumulators (512 columns).
+//   Per query tile the MMA thread issues S^T = K Q^T, dP^T = V dO^T,
+//   dV += P^T dO and dK += dS^T Q (the last two read P^T / dS^T from TMEM);
+//   it queues the next tile's S^T behind dV and the next dP^T behind dK, so
+//   the tensor core works while the four elementwise warps (one key row per
+//   thread) turn S^T into P^T and dP^T into dS^T.
+//
+// dQ: one CTA per (128-row query tile, query head, batch).  Q and dO stay in
+//   shared memory; K tiles stream through a three-stage ring and V tiles
+//   through a two-stage ring.  TMEM: two S buffers (scores, later dS as
+//   16-bit pairs), dP, and the dQ accumulator.  Per key tile: S = Q K^T,
+//   dP = dO V^T, then dQ += dS K; S for tile j+2 is queued behind dQ_j so the
+//   exponentials of one tile overlap the MMAs of the next.
+//
+// Every mbarrier wait is bounded (sm100.cuh) and the roles drain in-flight
+// copies and MMAs before tensor memory is released.
+#include <cuda.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kT = 128;        // rows of every tile (keys or queries) = TMEM lanes
+constexpr int kThreads = 192;  // warps 0-3 elementwise, 4 TMA, 5 MMA
+constexpr int kWarpLoad = 4;
+constexpr int kWarpMma = 5;
+constexpr int kPanel = 128 * 128;  // [128 rows][64 cols] 16-bit panel, bytes
+
+struct Params {
+  const float* lse;
+  const float* dvec;
+  void* out0;  // dK (dK/dV kernel) or dQ
+  void* out1;  // dV (dK/dV kernel)
+  int B, Hq, Hkv, Nq, Nk;
+  float scale;
+  float scale_log2;
+  int* status;
+};
+
+// Store one 128-byte-aligned row segment of D 16-bit values from fp32 TMEM columns.
+template <typename T, int D>
+__device__ __forceinline__ void store_row(uint32_t taddr, uint16_t* dst, float mul, bool valid) {
+#pragma unroll
+  for (int q = 0; q < D / 32; ++q) {
+    uint32_t r[32];
+    tmem_ld32(taddr + q * 32, r);
+    tmem_wait_ld();
+    reg_fence(r);
+    if (valid) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + q * 32);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        uint4 w;
+        w.x = Elem<T>::pack(__uint_as_float(r[8 * v + 0]) * mul, __uint_as_float(r[8 * v + 1]) * mul);
+        w.y = Elem<T>::pack(__uint_as_float(r[8 * v + 2]) * mul, __uint_as_float(r[8 * v + 3]) * mul);
+        w.z = Elem<T>::pack(__uint_as_float(r[8 * v + 4]) * mul, __uint_as_float(r[8 * v + 5]) * mul);
+        w.w = Elem<T>::pack(__uint_as_float(r[8 * v + 6]) * mul, __uint_as_float(r[8 * v + 7]) * mul);
+        d4[v] = w;
+      }
+    }
+  }
+}
+
+// 128 fp32 TMEM columns of this thread's lane into s[].
+__device__ __forceinline__ void load_row128(uint32_t taddr, float (&s)[kT]) {
+  uint32_t r0[32], r1[32], r2[32], r3[32];
+  tmem_ld32(taddr + 0, r0);
+  tmem_ld32(taddr + 32, r1);
+  tmem_ld32(taddr + 64, r2);
+  tmem_ld32(taddr + 96, r3);
+  tmem_wait_ld();
+  reg_fence(r0);
+  reg_fence(r1);
+  reg_fence(r2);
+  reg_fence(r3);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    s[i] = __uint_as_float(r0[i]);
+    s[32 + i] = __uint_as_float(r1[i]);
+    s[64 + i] = __uint_as_float(r2[i]);
+    s[96 + i] = __uint_as_float(r3[i]);
+  }
+}
+
+// dS = P (dP - d) column by column, written back as 16-bit pairs over the
+// first 64 columns starting at `tds`; reads dP 32 columns at a time from `tdp`.
+// When tds == tdp the writes trail the reads (columns 16c.. after 32c.. are read).
+template <typename T, bool PER_COL_D>
+__device__ __forceinline__ void write_ds(uint32_t tdp, uint32_t tds, const float (&p)[kT], const float* dcol,
+                                         float drow) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t r[32];
+    tmem_ld32(tdp + q * 32, r);
+    tmem_wait_ld();
+    reg_fence(r);
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c0 = q * 32 + 2 * i, c1 = c0 + 1;
+      const float d0 = PER_COL_D ? dcol[c0] : drow;
+      const float d1 = PER_COL_D ? dcol[c1] : drow;
+      pk[i] = Elem<T>::pack(p[c0] * (__uint_as_float(r[2 * i]) - d0), p[c1] * (__uint_as_float(r[2 * i + 1]) - d1));
+    }
+    tmem_st16(tds + q * 16, pk);
+  }
+}
+
+// ===========================================================================
+// dK / dV
+// ===========================================================================
+template <int D>
+struct DkdvSmem {
+  static constexpr int kTile = (D / 64) * kPanel;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kTile;
+  static constexpr int kOffQ = 2 * kTile;   // 2 stages
+  static constexpr int kOffDO = 4 * kTile;  // 2 stages
+  static constexpr int kOffLse = 6 * kTile;  // [2][128] fp32, log2 domain
+  static constexpr int kOffD = kOffLse + 2 * kT * 4;
+  static constexpr int kOffBar = kOffD + 2 * kT * 4;
+  enum { kBarKV = 0, kBarQFull = 1, kBarQEmpty = 3, kBarS = 5, kBarDP = 6, kBarP = 7, kBarDS = 8, kBarDone = 9,
+         kBarDrain = 10, kBarLse = 11, kNumBars = 13 };
+  static constexpr int kOffTmem = kOffBar + kNumBars * 8;
+  static constexpr int kOffAbort = kOffTmem + 4;
+  static constexpr int kBytes = kOffAbort + 4 + 1024;
+};
+// TMEM columns: S^T / P^T, dP^T / dS^T, dV, dK
+constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256, kColDK = 384;
+
+template <typename T, int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                          Params p) {
+  using L = DkdvSmem<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* gb = smem_raw + (sb - raw);
+  auto bar = [&](int i) { return sb + L::kOffBar + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + L::kOffAbort);
+  float* s_lse = reinterpret_cast<float*>(gb + L::kOffLse);
+  float* s_d = reinterpret_cast<float*>(gb + L::kOffD);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int kt = blockIdx.x;  // small key tiles see the most query tiles: launched first
+  const int hk = blockIdx.y, b = blockIdx.z;
+  const int G = p.Hq / p.Hkv;
+  const int k0 = kt * kT;
+  const int off = p.Nk - p.Nq;
+  const int mstart = CAUSAL ? max(0, k0 - off) / kT : 0;
+  const int nq = (p.Nq + kT - 1) / kT;
+  const int per_head = nq - mstart;
+  const int nt = G * per_head;  // query tiles this CTA visits
+
+  if (tid == 0) {
+    for (int i = 0; i < L::kNumBars; ++i)
+      mbar_init(bar(i), (i == L::kBarP || i == L::kBarDS || i >= L::kBarLse) ? kT : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(sb + L::kOffTmem, 512);
+    tmem_relinquish();
+  }
+  if (warp == kWarpLoad && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmDO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(gb + L::kOffTmem);
+
+  if (warp == kWarpLoad) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int last_u[2] = {-1, -1};
+      mbar_expect_tx(bar(L::kBarKV), 2 * L::kTile);
+#pragma unroll
+      for (int pn = 0; pn < D / 64; ++pn) {
+        tma_load_4d(sb + L::kOffK + pn * kPanel, &tmK, bar(L::kBarKV), 64 * pn, hk, k0, b);
+        tma_load_4d(sb + L::kOffV + pn * kPanel, &tmV, bar(L::kBarKV), 64 * pn, hk, k0, b);
+      }
+      for (int t = 0; t < nt; ++t) {
+        const int st = t & 1, u = t >> 1;
+        const int h = hk * G + t / per_head;
+        const int i0 = (mstart + t % per_head) * kT;
+        if (u > 0 && !mbar_wait(bar(L::kBarQEmpty + st), (u - 1) & 1, abort_flag, p.status)) break;
+        mbar_expect_tx(bar(L::kBarQFull + st), 2 * L::kTile);
+#pragma unroll
+        for (int pn = 0; pn < D / 64; ++pn) {
+          tma_load_4d(sb + L::kOffQ + st * L::kTile + pn * kPanel, &tmQ, bar(L::kBarQFull + st), 64 * pn, h, i0, b);
+          tma_load_4d(sb + L::kOffDO + st * L::kTile + pn * kPanel, &tmDO, bar(L::kBarQFull + st), 64 * pn, h, i0,
+                      b);
+        }
+        last_u[st] = u;
+      }
+      if (*abort_flag) {
+        wait_drain(bar(L::kBarKV), 0, p.status);
+        for (int st = 0; st < 2; ++st)
+          if (last_u[st] >= 0) wait_drain(bar(L::kBarQFull + st), last_u[st] & 1, p.status);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr bool kBf16 = Elem<T>::kBf16;
+      constexpr uint32_t id_kk = idesc_f16(kBf16, kT, kT, false);  // S^T, dP^T: both operands K(=d)-major
+      constexpr uint32_t id_mn = idesc_f16(kBf16, kT, D, true);    // dV, dK: B = [queries][d], d contiguous
+      auto kmajor = [&](uint32_t dst, uint32_t a_base, uint32_t b_base) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk >> 2) * kPanel + (kk & 3) * 32;
+          mma_ss(tbase + dst, sdesc_sw128(a_base + ko, 16, 1024), sdesc_sw128(b_base + ko, 16, 1024), id_kk,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      auto accum = [&](uint32_t dst, uint32_t a_col, uint32_t b_base, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < kT / 16; ++kk)
+          mma_ts(tbase + dst, tbase + a_col + kk * 8, sdesc_sw128(b_base + kk * 2048, kPanel, 1024), id_mn,
+                 (!first || kk > 0) ? 1u : 0u);
+      };
+      const uint32_t sK = sb + L::kOffK, sV = sb + L::kOffV;
+      auto sQ = [&](int st) { return sb + L::kOffQ + st * L::kTile; };
+      auto sDO = [&](int st) { return sb + L::kOffDO + st * L::kTile; };
+      bool ok = mbar_wait(bar(L::kBarKV), 0, abort_flag, p.status) &&
+                mbar_wait(bar(L::kBarQFull), 0, abort_flag, p.status);
+      if (ok) {
+        tc_fence_after();
+        kmajor(kColST, sK, sQ(0));
+        mma_commit(bar(L::kBarS));
+        kmajor(kColDPT, sV, sDO(0));
+        mma_commit(bar(L::kBarDP));
+        for (int t = 0; t < nt; ++t) {
+          const int st = t & 1;
+          const bool more = t + 1 < nt;
+          ok = mbar_wait(bar(L::kBarP), t & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc_fence_after();
+          accum(kColDV, kColST, sDO(st), t == 0);
+          if (more) {
+            ok = mbar_wait(bar(L::kBarQFull + (st ^ 1)), ((t + 1) >> 1) & 1, abort_flag, p.status);
+            if (!ok) break;
+            tc_fence_after();
+            kmajor(kColST, sK, sQ(st ^ 1));  // overwrites P^T after the dV MMA in issue order
+            mma_commit(bar(L::kBarS));
+          }
+          ok = mbar_wait(bar(L::kBarDS), t & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc_fence_after();
+          accum(kColDK, kColDPT, sQ(st), t == 0);
+          mma_commit(bar(L::kBarQEmpty + st));
+          if (more) {
+            kmajor(kColDPT, sV, sDO(st ^ 1));  // overwrites dS^T after the dK MMA in issue order
+            mma_commit(bar(L::kBarDP));
+          }
+        }
+        if (ok) mma_commit(bar(L::kBarDone));
+      }
+      mma_commit(bar(L::kBarDrain));
+      wait_drain(bar(L::kBarDrain), 0, p.status);
+    }
+  } else {
+    // ------------------------------------------------------------------ elementwise: one key row per thread
+    const int wq = warp;
+    const int jrow = wq * 32 + lane;
+    const int key = k0 + jrow;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tST = tbase + lane_off + kColST, tDPT = tbase + lane_off + kColDPT;
+    const float c = p.scale_log2;
+    auto fetch = [&](int t, float& lv, float& dv) {
+      const int h = hk * G + t / per_head;
+      const int i = (mstart + t % per_head) * kT + tid;
+      const long idx = ((long)b * p.Hq + h) * p.Nq + i;
+      lv = i < p.Nq ? p.lse[idx] * kLog2e : INFINITY;  // rows past Nq get P = 0
+      dv = i < p.Nq ? p.dvec[idx] : 0.f;
+    };
+    // LSE and D of query tile t sit in shared buffer t & 1; every elementwise thread
+    // writes one entry and arrives on kBarLse + buffer.  Waiting for buffer t & 1
+    // also proves every thread finished reading it in iteration t - 2.
+    {
+      float lv, dv;
+      fetch(0, lv, dv);
+      s_lse[tid] = lv;
+      s_d[tid] = dv;
+      mbar_arrive(bar(L::kBarLse));
+    }
+    bool ok = true;
+    for (int t = 0; t < nt; ++t) {
+      const int buf = t & 1;
+      const int i0 = (mstart + t % per_head) * kT;
+      float nl = 0.f, nd = 0.f;
+      if (t + 1 < nt) fetch(t + 1, nl, nd);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarLse + buf), (t >> 1) & 1, abort_flag, p.status));
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS), t & 1, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      float pv[kT];
+      load_row128(tST, pv);
+      const float* lse_t = s_lse + buf * kT;
+#pragma unroll
+      for (int cc = 0; cc < kT; ++cc) pv[cc] = ex2(fmaf(pv[cc], c, -lse_t[cc]));
+      if (CAUSAL && k0 + kT - 1 > i0 + off) {
+        const int lim = key - off - i0;  // queries i0 + cc with cc < lim cannot see this key
+#pragma unroll
+        for (int cc = 0; cc < kT; ++cc)
+          if (cc < lim) pv[cc] = 0.f;
+      }
+      {
+        uint32_t pk0[32], pk1[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          pk0[i] = Elem<T>::pack(pv[2 * i], pv[2 * i + 1]);
+          pk1[i] = Elem<T>::pack(pv[64 + 2 * i], pv[64 + 2 * i + 1]);
+        }
+        tmem_st32(tST + 0, pk0);
+        tmem_st32(tST + 32, pk1);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(L::kBarP));
+
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), t & 1, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      write_ds<T, true>(tDPT, tDPT, pv, s_d + buf * kT, 0.f);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(L::kBarDS));
+      if (t + 1 < nt) {
+        s_lse[(buf ^ 1) * kT + tid] = nl;
+        s_d[(buf ^ 1) * kT + tid] = nd;
+        mbar_arrive(bar(L::kBarLse + (buf ^ 1)));
+      }
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDone), 0, abort_flag, p.status));
+    if (ok) {
+      tc_fence_after();
+      const bool valid = key < p.Nk;
+      const long row = ((long)b * p.Nk + key) * p.Hkv + hk;
+      store_row<T, D>(tbase + lane_off + kColDV, static_cast<uint16_t*>(p.out1) + row * D, 1.f, valid);
+      store_row<T, D>(tbase + lane_off + kColDK, static_cast<uint16_t*>(p.out0) + row * D, p.scale, valid);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ===========================================================================
+// dQ
+// ===========================================================================
+template <int D>
+struct DqSmem {
+  static constexpr int kTile = (D / 64) * kPanel;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffDO = kTile;
+  static constexpr int kOffK = 2 * kTile;  // 3 stages
+  static constexpr int kOffV = 5 * kTile;  // 2 stages
+  static constexpr int kOffBar = 7 * kTile;
+  enum { kBarQ = 0, kBarKFull = 1, kBarKEmpty = 4, kBarVFull = 7, kBarVEmpty = 9, kBarS = 11, kBarDP = 13,
+         kBarDS = 14, kBarDone = 15, kBarDrain = 16, kNumBars = 17 };
+  static constexpr int kOffTmem = kOffBar + kNumBars * 8;
+  static constexpr int kOffAbort = kOffTmem + 4;
+  static constexpr int kBytes = kOffAbort + 4 + 1024;
+};
+// TMEM columns: S buffers (scores, later dS), dP, dQ
+__host__ __device__ constexpr uint32_t col_s(int buf) { return 128u * buf; }
+constexpr uint32_t kColDP = 256, kColDQ = 384;
+
+template <typename T, int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                        Params p) {
+  using L = DqSmem<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* gb = smem_raw + (sb - raw);
+  auto bar = [&](int i) { return sb + L::kOffBar + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + L::kOffAbort);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int mblk = CAUSAL ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;  // longest causal rows first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / (p.Hq / p.Hkv);
+  const int m0 = mblk * kT;
+  const int off = p.Nk - p.Nq;
+  const int n_end = CAUSAL ? min(p.Nk, m0 + kT + off) : p.Nk;
+  const int n = (n_end + kT - 1) / kT;
+
+  if (tid == 0) {
+    for (int i = 0; i < L::kNumBars; ++i) mbar_init(bar(i), i == L::kBarDS ? kT : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(sb + L::kOffTmem, 512);
+    tmem_relinquish();
+  }
+  if (warp == kWarpLoad && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmDO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(gb + L::kOffTmem);
+
+  if (warp == kWarpLoad) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int last_k[3] = {-1, -1, -1}, last_v[2] = {-1, -1};
+      mbar_expect_tx(bar(L::kBarQ), 2 * L::kTile);
+#pragma unroll
+      for (int pn = 0; pn < D / 64; ++pn) {
+        tma_load_4d(sb + L::kOffQ + pn * kPanel, &tmQ, bar(L::kBarQ), 64 * pn, h, m0, b);
+        tma_load_4d(sb + L::kOffDO + pn * kPanel, &tmDO, bar(L::kBarQ), 64 * pn, h, m0, b);
+      }
+      for (int j = 0; j < n; ++j) {
+        const int ks = j % 3, ku = j / 3, vs = j & 1, vu = j >> 1;
+        if (ku > 0 && !mbar_wait(bar(L::kBarKEmpty + ks), (ku - 1) & 1, abort_flag, p.status)) break;
+        mbar_expect_tx(bar(L::kBarKFull + ks), L::kTile);
+#pragma unroll
+        for (int pn = 0; pn < D / 64; ++pn)
+          tma_load_4d(sb + L::kOffK + ks * L::kTile + pn * kPanel, &tmK, bar(L::kBarKFull + ks), 64 * pn, hk, j * kT,
+                      b);
+        last_k[ks] = ku;
+        if (vu > 0 && !mbar_wait(bar(L::kBarVEmpty + vs), (vu - 1) & 1, abort_flag, p.status)) break;
+        mbar_expect_tx(bar(L::kBarVFull + vs), L::kTile);
+#pragma unroll
+        for (int pn = 0; pn < D / 64; ++pn)
+          tma_load_4d(sb + L::kOffV + vs * L::kTile + pn * kPanel, &tmV, bar(L::kBarVFull + vs), 64 * pn, hk, j * kT,
+                      b);
+        last_v[vs] = vu;
+      }
+      if (*abort_flag) {
+        wait_drain(bar(L::kBarQ), 0, p.status);
+        for (int s3 = 0; s3 < 3; ++s3)
+          if (last_k[s3] >= 0) wait_drain(bar(L::kBarKFull + s3), last_k[s3] & 1, p.status);
+        for (int s2 = 0; s2 < 2; ++s2)
+          if (last_v[s2] >= 0) wait_drain(bar(L::kBarVFull + s2), last_v[s2] & 1, p.status);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr bool kBf16 = Elem<T>::kBf16;
+      constexpr uint32_t id_kk = idesc_f16(kBf16, kT, kT, false);  // S, dP
+      constexpr uint32_t id_mn = idesc_f16(kBf16, kT, D, true);    // dQ: B = K as [keys][d]
+      auto kmajor = [&](uint32_t dst, uint32_t a_base, uint32_t b_base) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk >> 2) * kPanel + (kk & 3) * 32;
+          mma_ss(tbase + dst, sdesc_sw128(a_base + ko, 16, 1024), sdesc_sw128(b_base + ko, 16, 1024), id_kk,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      const uint32_t sQ = sb + L::kOffQ, sDO = sb + L::kOffDO;
+      auto sK = [&](int j) { return sb + L::kOffK + (j % 3) * L::kTile; };
+      auto sV = [&](int j) { return sb + L::kOffV + (j & 1) * L::kTile; };
+      auto issue_s = [&](int j) -> bool {
+        if (!mbar_wait(bar(L::kBarKFull + j % 3), (j / 3) & 1, abort_flag, p.status)) return false;
+        tc_fence_after();
+        kmajor(col_s(j & 1), sQ, sK(j));
+        mma_commit(bar(L::kBarS + (j & 1)));
+        return true;
+      };
+      auto issue_dp = [&](int j) -> bool {
+        if (!mbar_wait(bar(L::kBarVFull + (j & 1)), (j >> 1) & 1, abort_flag, p.status)) return false;
+        tc_fence_after();
+        kmajor(kColDP, sDO, sV(j));
+        mma_commit(bar(L::kBarDP));
+        mma_commit(bar(L::kBarVEmpty + (j & 1)));
+        return true;
+      };
+      bool ok = mbar_wait(bar(L::kBarQ), 0, abort_flag, p.status);
+      ok = ok && issue_s(0) && issue_dp(0);
+      if (ok && n > 1) ok = issue_s(1);
+      if (ok) {
+        for (int j = 0; j < n; ++j) {
+          ok = mbar_wait(bar(L::kBarDS), j & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kT / 16; ++kk)
+            mma_ts(tbase + kColDQ, tbase + col_s(j & 1) + kk * 8, sdesc_sw128(sK(j) + kk * 2048, kPanel, 1024), id_mn,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(L::kBarKEmpty + j % 3));
+          if (j + 1 < n && !(ok = issue_dp(j + 1))) break;  // dP_j was read before dS_j was signalled
+          if (j + 2 < n && !(ok = issue_s(j + 2))) break;   // reuses S buffer j after the dQ MMA
+        }
+        if (ok) mma_commit(bar(L::kBarDone));
+      }
+      mma_commit(bar(L::kBarDrain));
+      wait_drain(bar(L::kBarDrain), 0, p.status);
+    }
+  } else {
+    // ------------------------------------------------------------------ elementwise: one query row per thread
+    const int wq = warp;
+    const int row = m0 + wq * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const float c = p.scale_log2;
+    const long idx = ((long)b * p.Hq + h) * p.Nq + row;
+    const float lse2 = row < p.Nq ? p.lse[idx] * kLog2e : INFINITY;
+    const float drow = row < p.Nq ? p.dvec[idx] : 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const uint32_t tS = tbase + lane_off + col_s(j & 1);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + (j & 1)), (j >> 1) & 1, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      float pv[kT];
+      load_row128(tS, pv);
+#pragma unroll
+      for (int cc = 0; cc < kT; ++cc) pv[cc] = ex2(fmaf(pv[cc], c, -lse2));
+      const int kb = j * kT;
+      if (kb + kT > p.Nk || (CAUSAL && kb + kT - 1 > m0 + off)) {
+        int lim = p.Nk - kb;
+        if (CAUSAL) lim = min(lim, row + off + 1 - kb);
+#pragma unroll
+        for (int cc = 0; cc < kT; ++cc)
+          if (cc >= lim) pv[cc] = 0.f;
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), j & 1, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      write_ds<T, false>(tbase + lane_off + kColDP, tS, pv, nullptr, drow);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(L::kBarDS));
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDone), 0, abort_flag, p.status));
+    if (ok) {
+      tc_fence_after();
+      const long orow = ((long)b * p.Nq + row) * p.Hq + h;
+      store_row<T, D>(tbase + lane_off + kColDQ, static_cast<uint16_t*>(p.out0) + orow * D, p.scale, row < p.Nq);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+struct Maps {
+  CUtensorMap q, k, v, dO;
+};
+
+bool make_maps(Maps& m, const BwdArgs& a) {
+  const bool bf16 = a.bf16 != 0;
+  return make_map(&m.q, a.q, bf16, a.d, a.Hq, a.Nq, a.B, kT) && make_map(&m.k, a.k, bf16, a.d, a.Hkv, a.Nk, a.B, kT) &&
+         make_map(&m.v, a.v, bf16, a.d, a.Hkv, a.Nk, a.B, kT) &&
+         make_map(&m.dO, a.dout, bf16, a.d, a.Hq, a.Nq, a.B, kT);
+}
+
+Params params(const BwdArgs& a, void* out0, void* out1) {
+  return Params{a.lse, a.dvec, out0, out1, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, a.scale, a.scale * kLog2e, a.status};
+}
+
+template <typename T, int D, bool CAUSAL>
+cudaError_t launch_dkdv(const BwdArgs& a, cudaStream_t s) {
+  Maps m;
+  if (!make_maps(m, a)) return cudaErrorInvalidValue;
+  auto kern = bwd_dkdv_sm100_kernel<T, D, CAUSAL>;
+  const int smem = DkdvSmem<D>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.Nk + kT - 1) / kT, a.Hkv, a.B);
+  kern<<<grid, kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, params(a, a.dk, a.dv));
+  return cudaGetLastError();
+}
+
+template <typename T, int D, bool CAUSAL>
+cudaError_t launch_dq(const BwdArgs& a, cudaStream_t s) {
+  Maps m;
+  if (!make_maps(m, a)) return cudaErrorInvalidValue;
+  auto kern = bwd_dq_sm100_kernel<T, D, CAUSAL>;
+  const int smem = DqSmem<D>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.Nq + kT - 1) / kT, a.Hq, a.B);
+  kern<<<grid, kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, params(a, a.dq, nullptr));
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+#define FA_DISPATCH_SM100(FN, a, s)                                                                        \
+  do {                                                                                                     \
+    if (a.bf16) {                                                                                          \
+      if (a.d == 128) return a.causal ? FN<__nv_bfloat16, 128, true>(a, s) : FN<__nv_bfloat16, 128, false>(a, s); \
+      return a.causal ? FN<__nv_bfloat16, 64, true>(a, s) : FN<__nv_bfloat16, 64, false>(a, s);           \
+    }                                                                                                      \
+    if (a.d == 128) return a.causal ? FN<__half, 128, true>(a, s) : FN<__half, 128, false>(a, s);         \
+    return a.causal ? FN<__half, 64, true>(a, s) : FN<__half, 64, false>(a, s);                           \
+  } while (0)
+
+cudaError_t launch_bwd_dkdv_sm100(const BwdArgs& a, cudaStream_t s) { FA_DISPATCH_SM100(launch_dkdv, a, s); }
+cudaError_t launch_bwd_dq_sm100(const BwdArgs& a, cudaStream_t s) { FA_DISPATCH_SM100(launch_dq, a, s); }
+
+}  // namespace fa

@@ -104,14 +104,15 @@ static fa_status bwd_run(int steps, const void* q, const void* k, const void* v,
   for (const void* p : p16)
     if (p && !aligned16(p)) return FA_ERR_ALIGN;
   if (lse && !aligned4(lse)) return FA_ERR_ALIGN;
+  if ((dkdv || dqs) && !fa::tma_available()) return FA_ERR_CUDA;  // the driver lacks the tensor-map encoder
   fa::BwdArgs a{q, k, v, o, dout, lse, dq, dk, dv, static_cast<float*>(workspace), B, Hq, Hkv, Nq, Nk, d,
                 causal ? 1 : 0, scale, dt == FA_BF16 ? 1 : 0, status_ptr()};
   if (!a.status) return FA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaSuccess;
   if (pre) e = fa::launch_bwd_preprocess(a, s);
-  if (e == cudaSuccess && dkdv) e = fa::launch_bwd_dkdv(a, s);
-  if (e == cudaSuccess && dqs) e = fa::launch_bwd_dq(a, s);
+  if (e == cudaSuccess && dkdv) e = fa::launch_bwd_dkdv_sm100(a, s);
+  if (e == cudaSuccess && dqs) e = fa::launch_bwd_dq_sm100(a, s);
   return from_cuda(e);
 }
 

@@ -31,8 +31,6 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
-#include <mutex>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -75,20 +73,6 @@ struct Params {
   float scale_log2;
   int* status;
 };
-
-// Bounded wait that ignores the abort flag (used while draining on the error path).
-__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, int* status) {
-  volatile int never = 0;
-  return mbar_wait(bar, parity, &never, status);
-}
-
-// Compiler barrier: later uses of r[] must follow the preceding tcgen05.wait::ld.
-__device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
-#pragma unroll
-  for (int i = 0; i < 32; i += 8)
-    asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]),
-                 "+r"(r[i + 6]), "+r"(r[i + 7]));
-}
 
 template <typename T, int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -364,34 +348,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  });
-  return fn;
-}
-
-// 4-D map over a BSHD tensor [B][N][H][D]: innermost d, then head, then row, then batch.
-// Box: 64 columns (128 bytes, 128-byte swizzle) x 1 head x `rows` rows x 1 batch.
-bool make_map(CUtensorMap* m, const void* base, bool bf16, int D, int H, int N, int B, int rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)N * H * D * 2};
-  cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
-  cuuint32_t es[4] = {1, 1, 1, 1};
-  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
-                  const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <typename T, int D, bool CAUSAL>
 cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
@@ -418,7 +374,7 @@ cudaError_t launch_t(const AttnArgs& a, cudaStream_t s) {
 }  // namespace
 
 bool fwd_sm100_supported(const AttnArgs& a) {
-  return (a.d == 64 || a.d == 128) && encode_fn() != nullptr;
+  return (a.d == 64 || a.d == 128) && tma_available();
 }
 
 cudaError_t launch_fwd_sm100(const AttnArgs& a, cudaStream_t s) {

@@ -2,6 +2,7 @@
 // Arguments are validated by the C ABI in fa_api.cu before any launcher runs.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -62,13 +63,20 @@ struct CombineArgs {
   int bf16;
 };
 
+// TMA descriptors (tma.cu).  make_map: 4-D map over a BSHD tensor [B][N][H][D]
+// (innermost d, then head, row, batch); box = 64 columns (128 bytes, 128-byte
+// swizzle) x 1 head x `rows` rows x 1 batch.  Out-of-range rows read as zero.
+bool tma_available();
+bool make_map(CUtensorMap* m, const void* base, bool bf16, int D, int H, int N, int B, int rows);
+
 // Forward on tcgen05 / TMEM / TMA (warp-specialised), d = 128 and 64.
 cudaError_t launch_fwd_sm100(const AttnArgs& a, cudaStream_t s);
 bool fwd_sm100_supported(const AttnArgs& a);
 
 cudaError_t launch_bwd_preprocess(const BwdArgs& a, cudaStream_t s);
-cudaError_t launch_bwd_dkdv(const BwdArgs& a, cudaStream_t s);
-cudaError_t launch_bwd_dq(const BwdArgs& a, cudaStream_t s);
+// Backward dK/dV and dQ on tcgen05 / TMEM / TMA, d = 128 and 64.
+cudaError_t launch_bwd_dkdv_sm100(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_dq_sm100(const BwdArgs& a, cudaStream_t s);
 
 cudaError_t launch_decode_split(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_decode_combine(const CombineArgs& a, cudaStream_t s);
