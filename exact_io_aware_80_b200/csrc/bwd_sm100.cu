@@ -103,6 +103,7 @@ __device__ __forceinline__ void load_row128(uint32_t taddr, float (&s)[kT]) {
 
 // dS = P (dP - d) column by column, written back as 16-bit pairs over the
 // first 64 columns starting at `tds`; reads dP 32 columns at a time from `tdp`.
+// The caller passes d negated: per column (dcol[c] = -D_c) or per row (drow = -D_i).
 // When tds == tdp the writes trail the reads (columns 16c.. after 32c.. are read).
 template <typename T, bool PER_COL_D>
 __device__ __forceinline__ void write_ds(uint32_t tdp, uint32_t tds, const float (&p)[kT], const float* dcol,
@@ -116,10 +117,11 @@ __device__ __forceinline__ void write_ds(uint32_t tdp, uint32_t tds, const float
     uint32_t pk[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const int c0 = q * 32 + 2 * i, c1 = c0 + 1;
-      const float d0 = PER_COL_D ? dcol[c0] : drow;
-      const float d1 = PER_COL_D ? dcol[c1] : drow;
-      pk[i] = Elem<T>::pack(p[c0] * (__uint_as_float(r[2 * i]) - d0), p[c1] * (__uint_as_float(r[2 * i + 1]) - d1));
+      const int c0 = q * 32 + 2 * i;
+      const float2 nd = PER_COL_D ? reinterpret_cast<const float2*>(dcol)[c0 >> 1] : make_float2(drow, drow);
+      const float2 ds = __fmul2_rn(make_float2(p[c0], p[c0 + 1]),
+                                   __fadd2_rn(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), nd));
+      pk[i] = Elem<T>::pack(ds.x, ds.y);
     }
     tmem_st16(tds + q * 16, pk);
   }
@@ -163,8 +165,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* s_d = reinterpret_cast<float*>(gb + L::kOffD);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int kt = blockIdx.x;  // small key tiles see the most query tiles: launched first
-  const int hk = blockIdx.y, b = blockIdx.z;
+  // grid (Hkv, key tiles, B), dispatched x-fastest: small key tiles see the most
+  // query tiles, so every head's longest work starts first
+  const int kt = blockIdx.y;
+  const int hk = blockIdx.x, b = blockIdx.z;
   const int G = p.Hq / p.Hkv;
   const int k0 = kt * kT;
   const int off = p.Nk - p.Nq;
@@ -297,8 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int h = hk * G + t / per_head;
       const int i = (mstart + t % per_head) * kT + tid;
       const long idx = ((long)b * p.Hq + h) * p.Nq + i;
-      lv = i < p.Nq ? p.lse[idx] * kLog2e : INFINITY;  // rows past Nq get P = 0
-      dv = i < p.Nq ? p.dvec[idx] : 0.f;
+      lv = i < p.Nq ? -p.lse[idx] * kLog2e : -INFINITY;  // negated; rows past Nq get P = 0
+      dv = i < p.Nq ? -p.dvec[idx] : 0.f;                 // negated
     };
     // LSE and D of query tile t sit in shared buffer t & 1; every elementwise thread
     // writes one entry and arrives on kBarLse + buffer.  Waiting for buffer t & 1
@@ -323,9 +327,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       float pv[kT];
       load_row128(tST, pv);
-      const float* lse_t = s_lse + buf * kT;
+      const float2* nl2 = reinterpret_cast<const float2*>(s_lse + buf * kT);
+      const float2 c2 = make_float2(c, c);
 #pragma unroll
-      for (int cc = 0; cc < kT; ++cc) pv[cc] = ex2(fmaf(pv[cc], c, -lse_t[cc]));
+      for (int cc = 0; cc < kT; cc += 2) {
+        const float2 x = __ffma2_rn(make_float2(pv[cc], pv[cc + 1]), c2, nl2[cc >> 1]);
+        pv[cc] = ex2(x.x);
+        pv[cc + 1] = ex2(x.y);
+      }
       if (CAUSAL && k0 + kT - 1 > i0 + off) {
         const int lim = key - off - i0;  // queries i0 + cc with cc < lim cannot see this key
 #pragma unroll
@@ -413,8 +422,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + L::kOffAbort);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int mblk = CAUSAL ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;  // longest causal rows first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // grid (Hq, row tiles, B), dispatched x-fastest: longest causal rows first across all heads
+  const int mblk = CAUSAL ? (int)(gridDim.y - 1 - blockIdx.y) : (int)blockIdx.y;
+  const int h = blockIdx.x, b = blockIdx.z;
   const int hk = h / (p.Hq / p.Hkv);
   const int m0 = mblk * kT;
   const int off = p.Nk - p.Nq;
@@ -537,8 +547,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const float c = p.scale_log2;
     const long idx = ((long)b * p.Hq + h) * p.Nq + row;
-    const float lse2 = row < p.Nq ? p.lse[idx] * kLog2e : INFINITY;
-    const float drow = row < p.Nq ? p.dvec[idx] : 0.f;
+    const float nlse2 = row < p.Nq ? -p.lse[idx] * kLog2e : -INFINITY;  // rows past Nq get P = 0
+    const float ndrow = row < p.Nq ? -p.dvec[idx] : 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const uint32_t tS = tbase + lane_off + col_s(j & 1);
@@ -547,8 +557,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       float pv[kT];
       load_row128(tS, pv);
+      const float2 c2 = make_float2(c, c), nl2 = make_float2(nlse2, nlse2);
 #pragma unroll
-      for (int cc = 0; cc < kT; ++cc) pv[cc] = ex2(fmaf(pv[cc], c, -lse2));
+      for (int cc = 0; cc < kT; cc += 2) {
+        const float2 x = __ffma2_rn(make_float2(pv[cc], pv[cc + 1]), c2, nl2);
+        pv[cc] = ex2(x.x);
+        pv[cc + 1] = ex2(x.y);
+      }
       const int kb = j * kT;
       if (kb + kT > p.Nk || (CAUSAL && kb + kT - 1 > m0 + off)) {
         int lim = p.Nk - kb;
@@ -560,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), j & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
-      write_ds<T, false>(tbase + lane_off + kColDP, tS, pv, nullptr, drow);
+      write_ds<T, false>(tbase + lane_off + kColDP, tS, pv, nullptr, ndrow);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(L::kBarDS));
@@ -608,7 +623,7 @@ cudaError_t launch_dkdv(const BwdArgs& a, cudaStream_t s) {
   const int smem = DkdvSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.Nk + kT - 1) / kT, a.Hkv, a.B);
+  dim3 grid(a.Hkv, (a.Nk + kT - 1) / kT, a.B);
   kern<<<grid, kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, params(a, a.dk, a.dv));
   return cudaGetLastError();
 }
@@ -621,7 +636,7 @@ cudaError_t launch_dq(const BwdArgs& a, cudaStream_t s) {
   const int smem = DqSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.Nq + kT - 1) / kT, a.Hq, a.B);
+  dim3 grid(a.Hq, (a.Nq + kT - 1) / kT, a.B);
   kern<<<grid, kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, params(a, a.dq, nullptr));
   return cudaGetLastError();
 }

@@ -87,8 +87,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + L::kOffAbort);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int mblk = CAUSAL ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;  // longest causal rows first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // grid (Hq, row blocks, B): blocks are dispatched x-fastest, so every head's
+  // longest causal row block starts before any shorter one
+  const int mblk = CAUSAL ? (int)(gridDim.y - 1 - blockIdx.y) : (int)blockIdx.y;
+  const int h = blockIdx.x, b = blockIdx.z;
   const int hk = h / (p.Hq / p.Hkv);
   const int m0 = mblk * (kTiles * kBM);
   const int off = p.Nk - p.Nq;
@@ -263,13 +265,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kBN; ++i)
           if (i >= lim) s[i] = -INFINITY;
       }
-      float mx[4] = {s[0], s[1], s[2], s[3]};
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int i = 4; i < kBN; i += 4) {
-        mx[0] = fmaxf(mx[0], s[i]);
-        mx[1] = fmaxf(mx[1], s[i + 1]);
-        mx[2] = fmaxf(mx[2], s[i + 2]);
-        mx[3] = fmaxf(mx[3], s[i + 3]);
+      for (int i = 0; i < kBN; i += 8) {
+        mx[0] = max3(mx[0], s[i], s[i + 1]);
+        mx[1] = max3(mx[1], s[i + 2], s[i + 3]);
+        mx[2] = max3(mx[2], s[i + 4], s[i + 5]);
+        mx[3] = max3(mx[3], s[i + 6], s[i + 7]);
       }
       const float mxs = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
       const bool resc = mxs > m_ref + kRescaleThreshold;
@@ -278,17 +280,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       l *= corr;
       const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
       uint32_t pk0[32], pk1[32];
-      float rs0 = 0.f, rs1 = 0.f;
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(-mu, -mu);
+      float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float a0 = ex2(fmaf(s[2 * i], c, -mu)), a1 = ex2(fmaf(s[2 * i + 1], c, -mu));
-        const float b0 = ex2(fmaf(s[64 + 2 * i], c, -mu)), b1 = ex2(fmaf(s[64 + 2 * i + 1], c, -mu));
-        rs0 += a0 + a1;
-        rs1 += b0 + b1;
-        pk0[i] = Elem<T>::pack(a0, a1);
-        pk1[i] = Elem<T>::pack(b0, b1);
+        const float2 x0 = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), c2, nm2);
+        const float2 x1 = __ffma2_rn(make_float2(s[64 + 2 * i], s[64 + 2 * i + 1]), c2, nm2);
+        const float2 a = make_float2(ex2(x0.x), ex2(x0.y)), bb = make_float2(ex2(x1.x), ex2(x1.y));
+        rs0 = __fadd2_rn(rs0, a);
+        rs1 = __fadd2_rn(rs1, bb);
+        pk0[i] = Elem<T>::pack(a.x, a.y);
+        pk1[i] = Elem<T>::pack(bb.x, bb.y);
       }
-      l += rs0 + rs1;
+      l += (rs0.x + rs0.y) + (rs1.x + rs1.y);
       tmem_st32(tS + 0, pk0);
       tmem_st32(tS + 32, pk1);
       if (__any_sync(0xffffffffu, resc && j > 0)) {
@@ -360,7 +364,7 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   const int smem = Smem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.Nq + kTiles * kBM - 1) / (kTiles * kBM), a.Hq, a.B);
+  dim3 grid(a.Hq, (a.Nq + kTiles * kBM - 1) / (kTiles * kBM), a.B);
   kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }

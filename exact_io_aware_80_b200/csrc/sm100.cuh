@@ -178,6 +178,13 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
                  "+r"(r[i + 6]), "+r"(r[i + 7]));
 }
 
+// max(a, b, c) in one instruction (sm_100 three-input max).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Bounded wait that ignores the abort flag (used while draining on the error path).
 __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, int* status) {
   volatile int never = 0;
