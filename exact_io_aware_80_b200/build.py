@@ -45,7 +45,7 @@ def _compile(src: str, force: bool, extra) -> str:
     obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
     if not force and os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(src), _newest_header()):
         return obj
-    cmd = [nvcc()] + ARCH + FLAGS + list(extra) + ["-c", src, "-o", obj]
+    cmd = [nvcc()] + ARCH + FLAGS + list(extra) + os.environ.get("FA_NVCC_EXTRA", "").split() + ["-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed for {src}:\n{' '.join(cmd)}\n{r.stdout}\n{r.stderr}")

@@ -331,9 +331,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 c2 = make_float2(c, c);
 #pragma unroll
       for (int cc = 0; cc < kT; cc += 2) {
-        const float2 x = __ffma2_rn(make_float2(pv[cc], pv[cc + 1]), c2, nl2[cc >> 1]);
-        pv[cc] = ex2(x.x);
-        pv[cc + 1] = ex2(x.y);
+        const float2 x = exp2_pair(__ffma2_rn(make_float2(pv[cc], pv[cc + 1]), c2, nl2[cc >> 1]), cc >> 1);
+        pv[cc] = x.x;
+        pv[cc + 1] = x.y;
       }
       if (CAUSAL && k0 + kT - 1 > i0 + off) {
         const int lim = key - off - i0;  // queries i0 + cc with cc < lim cannot see this key
@@ -560,9 +560,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 c2 = make_float2(c, c), nl2 = make_float2(nlse2, nlse2);
 #pragma unroll
       for (int cc = 0; cc < kT; cc += 2) {
-        const float2 x = __ffma2_rn(make_float2(pv[cc], pv[cc + 1]), c2, nl2);
-        pv[cc] = ex2(x.x);
-        pv[cc + 1] = ex2(x.y);
+        const float2 x = exp2_pair(__ffma2_rn(make_float2(pv[cc], pv[cc + 1]), c2, nl2), cc >> 1);
+        pv[cc] = x.x;
+        pv[cc + 1] = x.y;
       }
       const int kb = j * kT;
       if (kb + kT > p.Nk || (CAUSAL && kb + kT - 1 > m0 + off)) {

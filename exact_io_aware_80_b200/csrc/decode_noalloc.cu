@@ -22,7 +22,7 @@
 
 #include <mutex>
 
-#include "../../include/fa.h"
+#include "fa.h"
 #include "kernels.h"
 
 namespace {

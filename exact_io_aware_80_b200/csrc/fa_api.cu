@@ -7,7 +7,7 @@
 
 #include <mutex>
 
-#include "../../include/fa.h"
+#include "fa.h"
 #include "kernels.h"
 
 namespace {

@@ -7,7 +7,10 @@
 // and running sum l, rescale the output accumulator when m grows, and divide
 // by l at the end; the N x N score matrix never reaches HBM.
 //
-// How it maps onto one B200 SM (one CTA per SM, 320 threads):
+// How it maps onto one B200 SM: a persistent grid of one CTA per SM (384
+// threads = 3 warpgroups) walks the (row block, head, batch) work tiles,
+// longest causal row blocks first; the next tile's Q/K/V loads and first
+// score MMAs overlap the current tile's epilogue.  Per work tile:
 //   * two 128-row query tiles Q0, Q1 share every K/V tile the CTA loads;
 //   * warp 8 (one thread) issues TMA loads: Q0/Q1 once, then 128-key K and V
 //     tiles into a two-stage shared-memory ring (128-byte swizzle);
@@ -31,6 +34,8 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -45,8 +50,14 @@ constexpr int kBN = 128;     // keys per K/V tile
 constexpr int kTiles = 2;    // query tiles per CTA
 constexpr int kStages = 2;   // K/V ring depth
 constexpr int kWarpLoad = 8;
-constexpr int kWarpMma = 9;
-constexpr int kThreads = 320;
+constexpr int kWarpMma = 9;   // warps 10 and 11 only complete the third warpgroup
+constexpr int kThreads = 384;
+// Register split: launched at 168 per thread (384 x 168 = 64512); the
+// load/MMA warpgroup drops to 104 and the two softmax warpgroups rise to 200
+// (2 x 128 x 200 + 128 x 104 = 64512).
+constexpr int kRegsSoftmax = 200;
+constexpr int kRegsControl = 104;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * 168, "register split exceeds the launch");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when m grows by more than 2^8
 __host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }        // S_t / P_t
 __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * t; }  // O_t
@@ -59,8 +70,10 @@ struct Smem {
   static constexpr int kOffK = kOffQ + kTiles * kTile;
   static constexpr int kOffV = kOffK + kStages * kTile;
   static constexpr int kOffBar = kOffV + kStages * kTile;
+  // kBarQ/kBarQEmpty: the query tiles of a work tile landed / may be replaced; kBarO: both
+  // tiles' last PV finished; kBarOFree + t: the epilogue of tile t has read O_t
   enum { kBarQ = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7, kBarS = 9, kBarP = 11, kBarO = 13,
-         kBarDrain = 14, kNumBars = 15 };
+         kBarDrain = 14, kBarQEmpty = 15, kBarOFree = 16, kNumBars = 18 };
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmem + 4;
   static constexpr int kBytes = kOffAbort + 4 + 1024;  // + slack to align the base to 1024 B
@@ -72,7 +85,32 @@ struct Params {
   int B, Hq, Hkv, Nq, Nk;
   float scale_log2;
   int* status;
+  int num_mblk;  // 256-row blocks per (b, h)
+  int num_work;  // num_mblk * Hq * B work tiles
 };
+
+// Work tile w of the persistent schedule: row block, query head, batch.  Causal
+// row blocks are enumerated longest first (all heads and batches of one length
+// together).  CTA i takes one tile per round k, snaking across the grid:
+// w = k G + i on even rounds and k G + (G - 1 - i) on odd ones, which balances
+// the decreasing tile lengths across SMs (work_index below).
+struct Work {
+  int mblk, hq, b;
+};
+__device__ __forceinline__ int work_index(int round) {
+  const int G = gridDim.x, i = blockIdx.x;
+  return round * G + ((round & 1) ? (G - 1 - i) : i);
+}
+template <bool CAUSAL>
+__device__ __forceinline__ Work work_at(const Params& p, int w) {
+  const int per_len = p.Hq * p.B;
+  const int r = w / per_len, rest = w % per_len;
+  Work x;
+  x.mblk = CAUSAL ? p.num_mblk - 1 - r : r;
+  x.hq = rest % p.Hq;
+  x.b = rest / p.Hq;
+  return x;
+}
 
 template <typename T, int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -87,18 +125,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + L::kOffAbort);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // grid (Hq, row blocks, B): blocks are dispatched x-fastest, so every head's
-  // longest causal row block starts before any shorter one
-  const int mblk = CAUSAL ? (int)(gridDim.y - 1 - blockIdx.y) : (int)blockIdx.y;
-  const int h = blockIdx.x, b = blockIdx.z;
-  const int hk = h / (p.Hq / p.Hkv);
-  const int m0 = mblk * (kTiles * kBM);
   const int off = p.Nk - p.Nq;
-  const int n_end = CAUSAL ? min(p.Nk, m0 + kTiles * kBM + off) : p.Nk;
-  const int nblk = (n_end + kBN - 1) / kBN;
+  auto blocks_of = [&](int mblk) {  // K/V tiles a row block visits (causal rows stop at their diagonal)
+    const int m0 = mblk * (kTiles * kBM);
+    const int n_end = CAUSAL ? min(p.Nk, m0 + kTiles * kBM + off) : p.Nk;
+    return (n_end + kBN - 1) / kBN;
+  };
 
   if (tid == 0) {
-    for (int i = 0; i < L::kNumBars; ++i) mbar_init(bar(i), (i == L::kBarP || i == L::kBarP + 1) ? kBM : 1);
+    for (int i = 0; i < L::kNumBars; ++i)
+      mbar_init(bar(i), (i == L::kBarP || i == L::kBarP + 1 || i == L::kBarOFree || i == L::kBarOFree + 1) ? kBM : 1);
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -117,38 +153,58 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(gb + L::kOffTmem);
 
-  if (warp == kWarpLoad) {
+  if (warp >= kWarpLoad) {
+   regs_decrease<kRegsControl>();
+   if (warp == kWarpLoad) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int last_u[kStages] = {-1, -1};
-      mbar_expect_tx(bar(L::kBarQ), kTiles * L::kTile);
+      int last_q = -1;
+      int g = 0;  // K/V tiles loaded so far by this CTA (ring position)
+      for (int wl = 0, w = work_index(0); w < p.num_work; w = work_index(++wl)) {
+        const Work x = work_at<CAUSAL>(p, w);
+        const int hk = x.hq / (p.Hq / p.Hkv);
+        const int m0 = x.mblk * (kTiles * kBM);
+        const int nblk = blocks_of(x.mblk);
+        // the previous tile's last score MMAs must have read Q before it is replaced
+        if (wl > 0 && !mbar_wait(bar(L::kBarQEmpty), (wl - 1) & 1, abort_flag, p.status)) break;
+        mbar_expect_tx(bar(L::kBarQ), kTiles * L::kTile);
 #pragma unroll
-      for (int t = 0; t < kTiles; ++t)
+        for (int t = 0; t < kTiles; ++t)
 #pragma unroll
-        for (int pn = 0; pn < D / 64; ++pn)
-          tma_load_4d(sb + L::kOffQ + t * L::kTile + pn * L::kPanel, &tmQ, bar(L::kBarQ), 64 * pn, h, m0 + t * kBM, b);
-      for (int j = 0; j < nblk; ++j) {
-        const int st = j & 1, u = j >> 1;
-        if (u > 0 && !mbar_wait(bar(L::kBarKEmpty + st), (u - 1) & 1, abort_flag, p.status)) break;
-        mbar_expect_tx(bar(L::kBarKFull + st), L::kTile);
+          for (int pn = 0; pn < D / 64; ++pn)
+            tma_load_4d(sb + L::kOffQ + t * L::kTile + pn * L::kPanel, &tmQ, bar(L::kBarQ), 64 * pn, x.hq,
+                        m0 + t * kBM, x.b);
+        last_q = wl;
+        bool stop = false;
+        for (int j = 0; j < nblk; ++j, ++g) {
+          const int st = g & 1, u = g >> 1;
+          if (u > 0 && !mbar_wait(bar(L::kBarKEmpty + st), (u - 1) & 1, abort_flag, p.status)) {
+            stop = true;
+            break;
+          }
+          mbar_expect_tx(bar(L::kBarKFull + st), L::kTile);
 #pragma unroll
-        for (int pn = 0; pn < D / 64; ++pn)
-          tma_load_4d(sb + L::kOffK + st * L::kTile + pn * L::kPanel, &tmK, bar(L::kBarKFull + st), 64 * pn, hk,
-                      j * kBN, b);
-        if (u > 0 && !mbar_wait(bar(L::kBarVEmpty + st), (u - 1) & 1, abort_flag, p.status)) {
-          last_u[st] = u;  // K of this use is in flight
-          break;
+          for (int pn = 0; pn < D / 64; ++pn)
+            tma_load_4d(sb + L::kOffK + st * L::kTile + pn * L::kPanel, &tmK, bar(L::kBarKFull + st), 64 * pn, hk,
+                        j * kBN, x.b);
+          if (u > 0 && !mbar_wait(bar(L::kBarVEmpty + st), (u - 1) & 1, abort_flag, p.status)) {
+            last_u[st] = u;  // K of this use is in flight
+            stop = true;
+            break;
+          }
+          mbar_expect_tx(bar(L::kBarVFull + st), L::kTile);
+#pragma unroll
+          for (int pn = 0; pn < D / 64; ++pn)
+            tma_load_4d(sb + L::kOffV + st * L::kTile + pn * L::kPanel, &tmV, bar(L::kBarVFull + st), 64 * pn, hk,
+                        j * kBN, x.b);
+          last_u[st] = u;
         }
-        mbar_expect_tx(bar(L::kBarVFull + st), L::kTile);
-#pragma unroll
-        for (int pn = 0; pn < D / 64; ++pn)
-          tma_load_4d(sb + L::kOffV + st * L::kTile + pn * L::kPanel, &tmV, bar(L::kBarVFull + st), 64 * pn, hk,
-                      j * kBN, b);
-        last_u[st] = u;
+        if (stop) break;
       }
       if (*abort_flag) {
         // let every copy this thread issued land before the CTA releases its shared memory
-        wait_drain(bar(L::kBarQ), 0, p.status);
+        if (last_q >= 0) wait_drain(bar(L::kBarQ), last_q & 1, p.status);
         for (int st = 0; st < kStages; ++st)
           if (last_u[st] >= 0) {
             wait_drain(bar(L::kBarKFull + st), last_u[st] & 1, p.status);
@@ -179,21 +235,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tbase + col_o(t), tbase + col_s(t) + kk * 8, bd, idv, (!first || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(bar(L::kBarQ), 0, abort_flag, p.status) &&
-                mbar_wait(bar(L::kBarKFull), 0, abort_flag, p.status);
-      if (ok) {
+      bool ok = true;
+      int g = 0;  // K/V tiles consumed so far by this CTA; S/P barriers complete once per tile
+      for (int wl = 0, w = work_index(0); ok && w < p.num_work; w = work_index(++wl)) {
+        const int nblk = blocks_of(work_at<CAUSAL>(p, w).mblk);
+        ok = mbar_wait(bar(L::kBarQ), wl & 1, abort_flag, p.status) &&
+             mbar_wait(bar(L::kBarKFull + (g & 1)), (g >> 1) & 1, abort_flag, p.status);
+        if (!ok) break;
         tc_fence_after();
-        qk(0, 0);
+        // the previous tile's last PV ran before these in issue order; its S/P buffers are free
+        qk(0, g & 1);
         mma_commit(bar(L::kBarS + 0));
-        qk(1, 0);
+        qk(1, g & 1);
         mma_commit(bar(L::kBarS + 1));
-        mma_commit(bar(L::kBarKEmpty + 0));
-        for (int j = 0; j < nblk; ++j) {
-          const int st = j & 1, u = j >> 1;
+        mma_commit(bar(L::kBarKEmpty + (g & 1)));
+        if (nblk == 1) mma_commit(bar(L::kBarQEmpty));
+        for (int j = 0; j < nblk; ++j, ++g) {
+          const int st = g & 1, u = g >> 1;
           const bool more = j + 1 < nblk;
-          const int st1 = (j + 1) & 1, u1 = (j + 1) >> 1;
+          const int st1 = (g + 1) & 1, u1 = (g + 1) >> 1;
           ok = mbar_wait(bar(L::kBarVFull + st), u & 1, abort_flag, p.status) &&
-               mbar_wait(bar(L::kBarP + 0), j & 1, abort_flag, p.status);
+               mbar_wait(bar(L::kBarP + 0), g & 1, abort_flag, p.status);
+          // the first PV of a tile overwrites O_0: the previous tile's epilogue must have read it
+          if (ok && j == 0 && wl > 0) ok = mbar_wait(bar(L::kBarOFree + 0), (wl - 1) & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
           pv(0, st, j == 0);
@@ -204,7 +268,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             qk(0, st1);  // overwrites S0/P0 after PV0 in issue order
             mma_commit(bar(L::kBarS + 0));
           }
-          ok = mbar_wait(bar(L::kBarP + 1), j & 1, abort_flag, p.status);
+          ok = mbar_wait(bar(L::kBarP + 1), g & 1, abort_flag, p.status);
+          if (ok && j == 0 && wl > 0) ok = mbar_wait(bar(L::kBarOFree + 1), (wl - 1) & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
           pv(1, st, j == 0);
@@ -213,6 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             qk(1, st1);
             mma_commit(bar(L::kBarS + 1));
             mma_commit(bar(L::kBarKEmpty + st1));
+            if (j + 2 == nblk) mma_commit(bar(L::kBarQEmpty));  // last score MMAs of this tile issued
           }
         }
         if (ok) mma_commit(bar(L::kBarO));
@@ -221,122 +287,136 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar(L::kBarDrain));
       wait_drain(bar(L::kBarDrain), 0, p.status);
     }
+   }
   } else {
+    regs_increase<kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax + epilogue
     const int t = warp >> 2;
     const int wq = warp & 3;
-    const int row_first = m0 + t * kBM;
-    const int row = row_first + wq * 32 + lane;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tbase + lane_off + col_s(t);
     const uint32_t tO = tbase + lane_off + col_o(t);
     const float c = p.scale_log2;
-    float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nblk; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + t), j & 1, abort_flag, p.status));
-      if (!ok) break;
-      tc_fence_after();
-      float s[kBN];
-      {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        tmem_ld32(tS + 0, r0);
-        tmem_ld32(tS + 32, r1);
-        tmem_ld32(tS + 64, r2);
-        tmem_ld32(tS + 96, r3);
-        tmem_wait_ld();
-        reg_fence(r0);
-        reg_fence(r1);
-        reg_fence(r2);
-        reg_fence(r3);
+    int g = 0;  // K/V tiles processed so far by this CTA
+    for (int wl = 0, w = work_index(0); ok && w < p.num_work; w = work_index(++wl)) {
+      const Work x = work_at<CAUSAL>(p, w);
+      const int h = x.hq, b = x.b;
+      const int m0 = x.mblk * (kTiles * kBM);
+      const int nblk = blocks_of(x.mblk);
+      const int row_first = m0 + t * kBM;
+      const int row = row_first + wq * 32 + lane;
+      float m_ref = -INFINITY, l = 0.f;
+        for (int j = 0; j < nblk; ++j, ++g) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + t), g & 1, abort_flag, p.status));
+        if (!ok) break;
+        tc_fence_after();
+        float s[kBN];
+        {
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          tmem_ld32(tS + 0, r0);
+          tmem_ld32(tS + 32, r1);
+          tmem_ld32(tS + 64, r2);
+          tmem_ld32(tS + 96, r3);
+          tmem_wait_ld();
+          reg_fence(r0);
+          reg_fence(r1);
+          reg_fence(r2);
+          reg_fence(r3);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s[i] = __uint_as_float(r0[i]);
-          s[32 + i] = __uint_as_float(r1[i]);
-          s[64 + i] = __uint_as_float(r2[i]);
-          s[96 + i] = __uint_as_float(r3[i]);
+          for (int i = 0; i < 32; ++i) {
+            s[i] = __uint_as_float(r0[i]);
+            s[32 + i] = __uint_as_float(r1[i]);
+            s[64 + i] = __uint_as_float(r2[i]);
+            s[96 + i] = __uint_as_float(r3[i]);
+          }
         }
-      }
-      const int kbase = j * kBN;
-      if (kbase + kBN > p.Nk || (CAUSAL && kbase + kBN - 1 > row_first + off)) {
-        int lim = p.Nk - kbase;
-        if (CAUSAL) lim = min(lim, row + off + 1 - kbase);
+        const int kbase = j * kBN;
+        if (kbase + kBN > p.Nk || (CAUSAL && kbase + kBN - 1 > row_first + off)) {
+          int lim = p.Nk - kbase;
+          if (CAUSAL) lim = min(lim, row + off + 1 - kbase);
 #pragma unroll
-        for (int i = 0; i < kBN; ++i)
-          if (i >= lim) s[i] = -INFINITY;
-      }
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          for (int i = 0; i < kBN; ++i)
+            if (i >= lim) s[i] = -INFINITY;
+        }
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int i = 0; i < kBN; i += 8) {
-        mx[0] = max3(mx[0], s[i], s[i + 1]);
-        mx[1] = max3(mx[1], s[i + 2], s[i + 3]);
-        mx[2] = max3(mx[2], s[i + 4], s[i + 5]);
-        mx[3] = max3(mx[3], s[i + 6], s[i + 7]);
-      }
-      const float mxs = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
-      const bool resc = mxs > m_ref + kRescaleThreshold;
-      const float corr = resc ? ex2(m_ref - mxs) : 1.f;
-      if (resc) m_ref = mxs;
-      l *= corr;
-      const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-      uint32_t pk0[32], pk1[32];
-      const float2 c2 = make_float2(c, c), nm2 = make_float2(-mu, -mu);
-      float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
+        for (int i = 0; i < kBN; i += 8) {
+          mx[0] = max3(mx[0], s[i], s[i + 1]);
+          mx[1] = max3(mx[1], s[i + 2], s[i + 3]);
+          mx[2] = max3(mx[2], s[i + 4], s[i + 5]);
+          mx[3] = max3(mx[3], s[i + 6], s[i + 7]);
+        }
+        const float mxs = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
+        const bool resc = mxs > m_ref + kRescaleThreshold;
+        const float corr = resc ? ex2(m_ref - mxs) : 1.f;
+        if (resc) m_ref = mxs;
+        l *= corr;
+        const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const float2 c2 = make_float2(c, c), nm2 = make_float2(-mu, -mu);
+        float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float2 x0 = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), c2, nm2);
-        const float2 x1 = __ffma2_rn(make_float2(s[64 + 2 * i], s[64 + 2 * i + 1]), c2, nm2);
-        const float2 a = make_float2(ex2(x0.x), ex2(x0.y)), bb = make_float2(ex2(x1.x), ex2(x1.y));
-        rs0 = __fadd2_rn(rs0, a);
-        rs1 = __fadd2_rn(rs1, bb);
-        pk0[i] = Elem<T>::pack(a.x, a.y);
-        pk1[i] = Elem<T>::pack(bb.x, bb.y);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const int c0 = 64 * half + 2 * i;
+            const float2 a = exp2_pair(__ffma2_rn(make_float2(s[c0], s[c0 + 1]), c2, nm2), 32 * half + i);
+            const float2 bb = exp2_pair(__ffma2_rn(make_float2(s[c0 + 2], s[c0 + 3]), c2, nm2), 32 * half + i + 1);
+            rs0 = __fadd2_rn(rs0, a);
+            rs1 = __fadd2_rn(rs1, bb);
+            pk[i] = Elem<T>::pack(a.x, a.y);
+            pk[i + 1] = Elem<T>::pack(bb.x, bb.y);
+          }
+          tmem_st32(tS + 32 * half, pk);
+        }
+        l += (rs0.x + rs0.y) + (rs1.x + rs1.y);
+        if (__any_sync(0xffffffffu, resc && j > 0)) {
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t r[32];
+            tmem_ld32(tO + q * 32, r);
+            tmem_wait_ld();
+            reg_fence(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * corr);
+            tmem_st32(tO + q * 32, r);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::kBarP + t));
       }
-      l += (rs0.x + rs0.y) + (rs1.x + rs1.y);
-      tmem_st32(tS + 0, pk0);
-      tmem_st32(tS + 32, pk1);
-      if (__any_sync(0xffffffffu, resc && j > 0)) {
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarO), wl & 1, abort_flag, p.status));
+      if (ok) {
+        tc_fence_after();
+        const bool valid = row < p.Nq;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        uint16_t* orow = static_cast<uint16_t*>(p.o) + (((long)b * p.Nq + row) * p.Hq + h) * D;
 #pragma unroll
         for (int q = 0; q < D / 32; ++q) {
           uint32_t r[32];
           tmem_ld32(tO + q * 32, r);
           tmem_wait_ld();
           reg_fence(r);
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * corr);
-          tmem_st32(tO + q * 32, r);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(L::kBarP + t));
-    }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarO), 0, abort_flag, p.status));
-    if (ok) {
-      tc_fence_after();
-      const bool valid = row < p.Nq;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      uint16_t* orow = static_cast<uint16_t*>(p.o) + (((long)b * p.Nq + row) * p.Hq + h) * D;
-#pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
-        uint32_t r[32];
-        tmem_ld32(tO + q * 32, r);
-        tmem_wait_ld();
-        reg_fence(r);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 w;
-            w.x = Elem<T>::pack(__uint_as_float(r[8 * v + 0]) * inv, __uint_as_float(r[8 * v + 1]) * inv);
-            w.y = Elem<T>::pack(__uint_as_float(r[8 * v + 2]) * inv, __uint_as_float(r[8 * v + 3]) * inv);
-            w.z = Elem<T>::pack(__uint_as_float(r[8 * v + 4]) * inv, __uint_as_float(r[8 * v + 5]) * inv);
-            w.w = Elem<T>::pack(__uint_as_float(r[8 * v + 6]) * inv, __uint_as_float(r[8 * v + 7]) * inv);
-            dst[v] = w;
+            for (int v = 0; v < 4; ++v) {
+              uint4 w;
+              w.x = Elem<T>::pack(__uint_as_float(r[8 * v + 0]) * inv, __uint_as_float(r[8 * v + 1]) * inv);
+              w.y = Elem<T>::pack(__uint_as_float(r[8 * v + 2]) * inv, __uint_as_float(r[8 * v + 3]) * inv);
+              w.z = Elem<T>::pack(__uint_as_float(r[8 * v + 4]) * inv, __uint_as_float(r[8 * v + 5]) * inv);
+              w.w = Elem<T>::pack(__uint_as_float(r[8 * v + 6]) * inv, __uint_as_float(r[8 * v + 7]) * inv);
+              dst[v] = w;
+            }
           }
         }
+        if (valid) p.lse[((long)b * p.Hq + h) * p.Nq + row] = l > 0.f ? (m_ref + lg2(l)) * kLn2 : -INFINITY;
+        // O_t has been read: the next tile's first PV may overwrite it
+        tc_fence_before();
+        mbar_arrive(bar(L::kBarOFree + t));
       }
-      if (valid) p.lse[((long)b * p.Hq + h) * p.Nq + row] = l > 0.f ? (m_ref + lg2(l)) * kLn2 : -INFINITY;
     }
   }
 
@@ -359,12 +439,16 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   if (!make_map(&mq, a.q, bf16, D, a.Hq, a.Nq, a.B, kBM) || !make_map(&mk, a.k, bf16, D, a.Hkv, a.Nk, a.B, kBN) ||
       !make_map(&mv, a.v, bf16, D, a.Hkv, a.Nk, a.B, kBN))
     return cudaErrorInvalidValue;
-  Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, a.scale * kLog2e, a.status};
+  const int num_mblk = (a.Nq + kTiles * kBM - 1) / (kTiles * kBM);
+  const long long num_work = (long long)num_mblk * a.Hq * a.B;
+  if (num_work > (1ll << 31) - 1) return cudaErrorInvalidValue;
+  Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, a.scale * kLog2e, a.status, num_mblk, (int)num_work};
   auto kern = fwd_sm100_kernel<T, D, CAUSAL>;
   const int smem = Smem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.Hq, (a.Nq + kTiles * kBM - 1) / (kTiles * kBM), a.B);
+  // persistent: one CTA per SM (the shared-memory footprint allows no more), looping over work tiles
+  const int grid = (int)std::min<long long>(num_work, device_sm_count());
   kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }

@@ -67,6 +67,8 @@ struct CombineArgs {
 // (innermost d, then head, row, batch); box = 64 columns (128 bytes, 128-byte
 // swizzle) x 1 head x `rows` rows x 1 batch.  Out-of-range rows read as zero.
 bool tma_available();
+// Streaming multiprocessors of the current device (148 if the query fails).
+int device_sm_count();
 bool make_map(CUtensorMap* m, const void* base, bool bf16, int D, int H, int N, int B, int rows);
 
 // Forward on tcgen05 / TMEM / TMA (warp-specialised), d = 128 and 64.

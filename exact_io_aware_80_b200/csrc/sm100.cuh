@@ -178,11 +178,62 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
                  "+r"(r[i + 6]), "+r"(r[i + 7]));
 }
 
+// Warpgroup register split: every warp of a warpgroup executes the same one.
+// The block's launch total (threads x registers at launch) must cover the sum
+// of the new per-warpgroup counts, or the increase would wait forever.
+template <int N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // max(a, b, c) in one instruction (sm_100 three-input max).
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// 2^x on the FMA and integer pipes, for two values at once (x <= 8; x below
+// -126 is clamped, giving ~2^-126 instead of 0).  Range reduction: n =
+// round(x) by adding the 1.5 * 2^23 shifter, f = x - n in [-1/2, 1/2].  2^f by
+// a degree-3 minimax polynomial (Remez exchange; relative error 7.5e-5;
+// coefficients from gen_exp2_poly.py), then 2^n by adding n << 23 to the bits
+// of p(f): the shifted sum t = x + 1.5 * 2^23 holds n in its low bits, so
+// (bits(t) << 23) == n << 23 modulo 2^32.  The kernels use it for a fixed
+// share of the exponentials so that the multi-function unit (ex2.approx) and
+// the FMA pipe share the softmax work.
+constexpr float kExp2C0 = 9.999280572e-01f;
+constexpr float kExp2C1 = 6.932609677e-01f;
+constexpr float kExp2C2 = 2.426111251e-01f;
+constexpr float kExp2C3 = 5.517166853e-02f;
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  q = __ffma2_rn(q, f, make_float2(kExp2C1, kExp2C1));
+  q = __ffma2_rn(q, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
+// Of every four column pairs, how many take exp2_fma2 instead of ex2.approx.
+#ifndef FA_EXP2_FMA_PAIRS
+#define FA_EXP2_FMA_PAIRS 1
+#endif
+constexpr int kExp2FmaPairs = FA_EXP2_FMA_PAIRS;
+
+// 2^x for a pair of columns, routed by the pair's index (a constant once the
+// caller's loop is unrolled, so the branch folds away).
+__device__ __forceinline__ float2 exp2_pair(float2 x, int pair) {
+  if ((pair & 3) >= 4 - kExp2FmaPairs) return exp2_fma2(x);
+  return make_float2(ex2(x.x), ex2(x.y));
 }
 
 // Bounded wait that ignores the abort flag (used while draining on the error path).

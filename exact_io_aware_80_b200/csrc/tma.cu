@@ -29,6 +29,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 bool tma_available() { return encode_fn() != nullptr; }
 
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+      n > 0)
+    return n;
+  return 148;
+}
+
 bool make_map(CUtensorMap* m, const void* base, bool bf16, int D, int H, int N, int B, int rows) {
   auto fn = encode_fn();
   if (!fn) return false;
