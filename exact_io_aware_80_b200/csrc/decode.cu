@@ -7,7 +7,7 @@
 // Partial pass: one CTA per (split s, KV head h_kv, sequence b).  The
 // Hq/Hkv query rows of the GQA group share every K/V byte the CTA reads, so
 // the KV cache crosses HBM exactly once.  K/V tiles of 64 keys stream through
-// a four-stage cp.async ring; each of the four warps takes 16 keys of every
+// a three-stage cp.async ring (two CTAs per SM); each of the four warps takes 16 keys of every
 // tile, keeps its own running (m, l, O) for the group's rows, and the warps
 // are merged through shared memory at the end.  The group's rows (padded to
 // the 16-row MMA shape) multiply the tiles on the tensor cores; the pass is
@@ -22,11 +22,11 @@ namespace {
 
 constexpr int kThreads = 128;
 constexpr int kTileN = 64;
-constexpr int kStages = 4;
+constexpr int kStages = 3;  // 3 x 32 KB K/V stages: two CTAs fit on an SM
 constexpr int kRows = 16;  // MMA rows; the group's query heads, zero-padded
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(DecodeArgs p) {
+__global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(DecodeArgs p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   constexpr int kTile = kTileN * D * 2;
   const uint32_t sQ = smem_u32(smem);

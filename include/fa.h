@@ -113,9 +113,10 @@ fa_status fa_bwd_dq(const void* q, const void* k, const void* v, const void* o, 
                     fa_dtype dt, fa_stream_t stream);
 
 /*
- * Suggested number of key splits for fa_decode_splitkv: enough (b, h_kv, split)
- * units to fill `num_sms` SMs several times over (num_sms <= 0: query the
- * current device).  Always >= 1 and <= ceil(Nk_max / 64).
+ * Suggested number of key splits for fa_decode_splitkv: about 26 (b, h_kv, split)
+ * units per SM so that ragged sequence lengths even out (num_sms <= 0: query
+ * the current device), splits of at least 256 keys.  Always >= 1 and
+ * <= ceil(Nk_max / 64).
  */
 int fa_decode_num_splits(int B, int Hkv, int Nk_max, int d, int num_sms);
 
