@@ -24,9 +24,11 @@
  *  - GQA: Hq % Hkv == 0; query head h reads KV head h / (Hq / Hkv).
  *  - d must be 64 or 128 (FA_ERR_UNSUPPORTED otherwise).  Nq, Nk >= 1, any
  *    value (ragged tails are masked inside the kernels).
- *  - Every pointer is a DEVICE pointer, 16-byte aligned (FA_ERR_ALIGN).  The
+ *  - Every pointer is a DEVICE pointer; tensors and workspaces 16-byte
+ *    aligned, lse and seqlens_k 4-byte aligned (FA_ERR_ALIGN otherwise).  The
  *    caller owns and allocates every buffer, workspaces included; the library
- *    never allocates device memory and keeps no per-call state.
+ *    allocates no device memory and keeps no per-call state (fa_decode_noalloc
+ *    uses a fixed static array inside the library instead of a workspace).
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *    default stream).  The return value reports argument validation (checked
  *    before anything is launched) and launch errors only.  Errors raised by a
@@ -92,9 +94,9 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  * The three launches fa_bwd makes, callable one by one (same arguments, same
  * validation), so that a caller can time or schedule them separately:
  *   fa_bwd_preprocess: workspace D[b,h,i] = sum_c dout[b,i,h,c] * o[b,i,h,c] (fp32);
- *   fa_bwd_dkdv: dk, dv from q, k, v, dout, lse and D (one CTA per 64-key tile
+ *   fa_bwd_dkdv: dk, dv from q, k, v, dout, lse and D (one CTA per 128-key tile
  *     of a KV head, looping over its group's query heads and query tiles);
- *   fa_bwd_dq: dq from q, k, v, dout, lse and D (one CTA per 64-row query tile).
+ *   fa_bwd_dq: dq from q, k, v, dout, lse and D (one CTA per 128-row query tile).
  * fa_bwd_dkdv and fa_bwd_dq read the D that fa_bwd_preprocess wrote, so on one
  * stream the preprocess call must come first.  Arguments a step does not read
  * may be NULL (preprocess: q, k, v, lse, dq, dk, dv; dkdv: o, dq; dq: o, dk, dv).
