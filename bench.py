@@ -157,13 +157,19 @@ def barrier(torch, world):
         dist.barrier()
 
 
-def max_over_ranks(torch, world, x: float) -> float:
+def max_over_ranks(torch, world, x: float, device="cuda") -> float:
+    """The slowest rank's value (timings are reported as the max over ranks)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world, flops_per_rank, ms_per_step_max):
+    """Whole-job TFLOP/s: every rank runs the same per-GPU work (weak scaling)."""
+    return world * flops_per_rank / (ms_per_step_max * 1e-3) / 1e12
 
 
 # ---------------------------------------------------------------------------
@@ -243,7 +249,7 @@ def run_ours(args):
 
     F = attn_flops(B, Hq, N, N, d, True)
     ms_step = ms_max / K
-    value = world * (F * 3.5) / (ms_step * 1e-3) / 1e12
+    value = job_throughput(world, F * 3.5, ms_step)
     fwd_tflops = F / (per["fwd"] * 1e-3) / 1e12
     bwd_ms = per["bwd_preprocess"] + per["bwd_dkdv"] + per["bwd_dq"]
     bwd_tflops = 2.5 * F / (bwd_ms * 1e-3) / 1e12

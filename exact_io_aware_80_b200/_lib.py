@@ -40,6 +40,7 @@ SIGNATURES = {
     "fa_decode_chunk": (_I, [_I, _I]),
     "fa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "fa_get_device_status": (_I, [_P]),
+    "fa_watchdog_selftest": (_I, [_I, _P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
 }
@@ -128,6 +129,10 @@ def fa_decode_splitkv(q, k_cache, v_cache, seqlens_k, B, Hq, Hkv, Nk_max, d, sca
 def fa_decode_combine(workspace, o, lse, seqlens_k, B, Hq, num_splits, d, dt, stream):
     return _check("fa_decode_combine", load().fa_decode_combine(workspace, o, lse, seqlens_k, B, Hq, num_splits, d,
                                                                 dt, stream))
+
+
+def fa_watchdog_selftest(limit_us, stream):
+    return _check("fa_watchdog_selftest", load().fa_watchdog_selftest(limit_us, stream))
 
 
 def fa_get_device_status(stream):

@@ -228,6 +228,13 @@ fa_status fa_decode_combine(const void* workspace, void* o, float* lse, const in
   return from_cuda(fa::launch_decode_combine(a, static_cast<cudaStream_t>(stream)));
 }
 
+fa_status fa_watchdog_selftest(int limit_us, fa_stream_t stream) {
+  if (limit_us < 1 || limit_us > 2000000) return FA_ERR_INVALID;
+  int* st = status_ptr();
+  if (!st) return FA_ERR_CUDA;
+  return from_cuda(fa::launch_watchdog_selftest(st, limit_us, static_cast<cudaStream_t>(stream)));
+}
+
 fa_status fa_get_device_status(fa_stream_t stream) {
   int* p = status_ptr();
   if (!p) return FA_ERR_CUDA;

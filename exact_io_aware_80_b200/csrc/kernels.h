@@ -81,6 +81,8 @@ cudaError_t launch_bwd_dkdv_sm100(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_dq_sm100(const BwdArgs& a, cudaStream_t s);
 
 cudaError_t launch_decode_split(const DecodeArgs& a, cudaStream_t s);
+// One CTA waiting on a barrier nothing arrives on, limit in microseconds (watchdog.cu).
+cudaError_t launch_watchdog_selftest(int* status, int limit_us, cudaStream_t s);
 cudaError_t launch_decode_combine(const CombineArgs& a, cudaStream_t s);
 
 }  // namespace fa

@@ -45,8 +45,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of `bar`; false if the CTA aborted or the limit ran out.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
+// Wait for phase `parity` of `bar`; false if the CTA aborted or the limit
+// (SM clock cycles) ran out.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                          long long limit = kSpinLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   uint32_t n = 0;
@@ -54,7 +56,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_try_wait(bar, parity)) return true;
     if ((++n & 31u) == 0) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kSpinLimitCycles) {
+      if (clock64() - t0 > limit) {
         *abort_flag = 1;
         atomicCAS(status, 0, kStatusTimeout);
         return false;

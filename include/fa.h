@@ -191,6 +191,15 @@ fa_status fa_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
  */
 fa_status fa_get_device_status(fa_stream_t stream);
 
+/*
+ * Self-test of the kernels' failure detection, with no fault involved: launches
+ * one CTA that waits on an mbarrier nothing ever arrives on, through the same
+ * bounded-wait routine the attention kernels use, giving up after `limit_us`
+ * microseconds (1 .. 2000000).  A following fa_get_device_status must return
+ * FA_ERR_TIMEOUT, and the CUDA context stays usable.
+ */
+fa_status fa_watchdog_selftest(int limit_us, fa_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* fa_status_string(fa_status s);
 

@@ -281,3 +281,19 @@ def test_bitwise_determinism(fa):
     r2 = fa.decode(qd.cuda(), kc.cuda(), vc.cuda(), sl.cuda())
     assert torch.equal(r1[0], r2[0]) and torch.equal(r1[1], r2[1])
     assert fa.device_status() == 0
+
+
+def test_watchdog_times_out_cleanly_and_context_survives(fa):
+    """A bounded wait on a barrier nothing arrives on reports FA_ERR_TIMEOUT
+    through the status word (no trap, no hang), which then reads clean again,
+    and the next attention call works."""
+    from exact_io_aware_80_b200 import _lib
+    stream = torch.cuda.current_stream().cuda_stream
+    assert fa.device_status() == 0
+    _lib.fa_watchdog_selftest(20000, stream)  # 20 ms limit
+    assert fa.device_status() == _lib.FA_ERR_TIMEOUT
+    assert fa.device_status() == 0
+    q, k, v = workloads.make_inputs(1, 2, 2, 200, 200, 128, torch.bfloat16, seed_base=9)
+    o, lse = run_fwd(fa, q, k, v, True)
+    O, L = oracle.attention_fwd(f64(q), f64(k), f64(v), True, 1 / math.sqrt(128))
+    assert np.abs(o - O).max() <= O_TOL
