@@ -69,14 +69,18 @@ struct Smem {
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kTiles * kTile;
   static constexpr int kOffV = kOffK + kStages * kTile;
-  static constexpr int kOffBar = kOffV + kStages * kTile;
-  // kBarQ/kBarQEmpty: the query tiles of a work tile landed / may be replaced; kBarO: both
-  // tiles' last PV finished; kBarOFree + t: the epilogue of tile t has read O_t
+  static constexpr int kOffStage = kOffV + kStages * kTile;  // one 16-bit O tile on its way to a TMA store
+  static constexpr int kOffBar = kOffStage + kTile;
+  // kBarQ/kBarQEmpty: the query tiles of a work tile landed / may be replaced; kBarO + t: tile t's
+  // last PV finished; kBarOFree + t: the epilogue of tile t has read O_t from TMEM;
+  // kBarStageFull + t: tile t's rows are in the stage buffer; kBarStageDone + t: the TMA store of
+  // tile t has read the stage buffer (the two tiles take turns with it)
   enum { kBarQ = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7, kBarS = 9, kBarP = 11, kBarO = 13,
-         kBarDrain = 14, kBarQEmpty = 15, kBarOFree = 16, kNumBars = 18 };
+         kBarDrain = 15, kBarQEmpty = 16, kBarOFree = 17, kBarStageFull = 19, kBarStageDone = 21, kNumBars = 23 };
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmem + 4;
   static constexpr int kBytes = kOffAbort + 4 + 1024;  // + slack to align the base to 1024 B
+  static_assert(kBytes <= 232448, "shared memory per CTA exceeded");
 };
 
 struct Params {
@@ -115,7 +119,7 @@ __device__ __forceinline__ Work work_at(const Params& p, int w) {
 template <typename T, int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, Params p) {
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, Params p) {
   using L = Smem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -134,7 +138,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < L::kNumBars; ++i)
-      mbar_init(bar(i), (i == L::kBarP || i == L::kBarP + 1 || i == L::kBarOFree || i == L::kBarOFree + 1) ? kBM : 1);
+      mbar_init(bar(i), (i == L::kBarP || i == L::kBarP + 1 || i == L::kBarOFree || i == L::kBarOFree + 1 ||
+                         i == L::kBarStageFull || i == L::kBarStageFull + 1)
+                            ? kBM
+                            : 1);
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -147,6 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
+    prefetch_tmap(&tmO);
   }
   tc_fence_before();
   __syncthreads();
@@ -261,6 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           pv(0, st, j == 0);
+          if (!more) mma_commit(bar(L::kBarO + 0));
           if (more) {
             ok = mbar_wait(bar(L::kBarKFull + st1), u1 & 1, abort_flag, p.status);
             if (!ok) break;
@@ -273,6 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           pv(1, st, j == 0);
+          if (!more) mma_commit(bar(L::kBarO + 1));
           mma_commit(bar(L::kBarVEmpty + st));
           if (more) {
             qk(1, st1);
@@ -281,7 +291,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (j + 2 == nblk) mma_commit(bar(L::kBarQEmpty));  // last score MMAs of this tile issued
           }
         }
-        if (ok) mma_commit(bar(L::kBarO));
       }
       // no MMA may still run when TMEM is released
       mma_commit(bar(L::kBarDrain));
@@ -387,37 +396,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(L::kBarP + t));
       }
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarO), wl & 1, abort_flag, p.status));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarO + t), wl & 1, abort_flag, p.status));
+      uint32_t r[D];
       if (ok) {
+        // O_t: TMEM -> registers, then hand the TMEM columns back to the MMA thread at once
         tc_fence_after();
-        const bool valid = row < p.Nq;
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        uint16_t* orow = static_cast<uint16_t*>(p.o) + (((long)b * p.Nq + row) * p.Hq + h) * D;
 #pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
-          uint32_t r[32];
-          tmem_ld32(tO + q * 32, r);
-          tmem_wait_ld();
-          reg_fence(r);
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+        for (int q = 0; q < D / 32; ++q) tmem_ld32(tO + q * 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * q));
+        tmem_wait_ld();
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 w;
-              w.x = Elem<T>::pack(__uint_as_float(r[8 * v + 0]) * inv, __uint_as_float(r[8 * v + 1]) * inv);
-              w.y = Elem<T>::pack(__uint_as_float(r[8 * v + 2]) * inv, __uint_as_float(r[8 * v + 3]) * inv);
-              w.z = Elem<T>::pack(__uint_as_float(r[8 * v + 4]) * inv, __uint_as_float(r[8 * v + 5]) * inv);
-              w.w = Elem<T>::pack(__uint_as_float(r[8 * v + 6]) * inv, __uint_as_float(r[8 * v + 7]) * inv);
-              dst[v] = w;
-            }
-          }
-        }
-        if (valid) p.lse[((long)b * p.Hq + h) * p.Nq + row] = l > 0.f ? (m_ref + lg2(l)) * kLn2 : -INFINITY;
-        // O_t has been read: the next tile's first PV may overwrite it
+        for (int q = 0; q < D / 32; ++q) reg_fence(*reinterpret_cast<uint32_t(*)[32]>(r + 32 * q));
         tc_fence_before();
         mbar_arrive(bar(L::kBarOFree + t));
+        // the stage buffer alternates tile 0, tile 1, tile 0 (next work tile), ...
+        if (t == 1)
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarStageDone + 0), wl & 1, abort_flag, p.status));
+        else if (wl > 0)
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarStageDone + 1), (wl - 1) & 1, abort_flag, p.status));
+      }
+      if (ok) {
+        // O / l as 16-bit into the stage buffer, laid out as the TMA box expects: 64-column
+        // panels of 128-byte rows, 16-byte chunk c of row r at chunk c ^ (r & 7)
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const int rr = wq * 32 + lane;
+        const uint32_t srow = sb + L::kOffStage + rr * 128;
+        auto o2 = [&](int i) { return Elem<T>::pack(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv); };
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c)
+          st_shared_v4(srow + (c >> 3) * L::kPanel + (((c & 7) ^ (rr & 7)) << 4), o2(8 * c), o2(8 * c + 2),
+                       o2(8 * c + 4), o2(8 * c + 6));
+        fence_proxy_async_smem();
+        mbar_arrive(bar(L::kBarStageFull + t));
+        if (row < p.Nq) p.lse[((long)b * p.Hq + h) * p.Nq + row] = l > 0.f ? (m_ref + lg2(l)) * kLn2 : -INFINITY;
+        if (wq == 0 && lane == 0) {
+          // one thread of the tile stores it; rows past Nq are clipped by the tensor map
+          ok = mbar_wait(bar(L::kBarStageFull + t), wl & 1, abort_flag, p.status);
+          if (ok) {
+#pragma unroll
+            for (int pn = 0; pn < D / 64; ++pn)
+              tma_store_4d(&tmO, sb + L::kOffStage + pn * L::kPanel, 64 * pn, h, row_first, b);
+            bulk_commit();
+            bulk_wait_read_all();
+            mbar_arrive(bar(L::kBarStageDone + t));
+          }
+        }
+        ok = __all_sync(0xffffffffu, ok);
       }
     }
+    // stores must be complete before the CTA exits
+    if (wq == 0 && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -434,10 +461,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 template <typename T, int D, bool CAUSAL>
 cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   const bool bf16 = Elem<T>::kBf16;
   if (!make_map(&mq, a.q, bf16, D, a.Hq, a.Nq, a.B, kBM) || !make_map(&mk, a.k, bf16, D, a.Hkv, a.Nk, a.B, kBN) ||
-      !make_map(&mv, a.v, bf16, D, a.Hkv, a.Nk, a.B, kBN))
+      !make_map(&mv, a.v, bf16, D, a.Hkv, a.Nk, a.B, kBN) || !make_map(&mo, a.o, bf16, D, a.Hq, a.Nq, a.B, kBM))
     return cudaErrorInvalidValue;
   const int num_mblk = (a.Nq + kTiles * kBM - 1) / (kTiles * kBM);
   const long long num_work = (long long)num_mblk * a.Hq * a.B;
@@ -449,7 +476,7 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   // persistent: one CTA per SM (the shared-memory footprint allows no more), looping over work tiles
   const int grid = (int)std::min<long long>(num_work, device_sm_count());
-  kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, p);
+  kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mo, p);
   return cudaGetLastError();
 }
 
