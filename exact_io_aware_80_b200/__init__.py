@@ -14,15 +14,17 @@ from __future__ import annotations
 import math
 
 from . import _lib
-from ._lib import (FAError, fa_bwd, fa_bwd_dkdv, fa_bwd_dq, fa_bwd_preprocess, fa_bwd_workspace_bytes, fa_decode_chunk, fa_decode_combine,  # noqa: F401
-                   fa_decode_num_splits, fa_decode_splitkv, fa_decode_workspace_bytes, fa_fwd,
-                   fa_get_device_status, fa_version)
+from ._lib import (FAError, fa_bwd, fa_bwd_dkdv, fa_bwd_dq, fa_bwd_preprocess, fa_bwd_workspace_bytes,  # noqa: F401
+                   fa_decode_chunk, fa_decode_combine, fa_decode_num_splits, fa_decode_splitkv,
+                   fa_decode_workspace_bytes, fa_fp8_quantize_qk, fa_fp8_quantize_v, fa_fp8_v_workspace_bytes, fa_fwd,
+                   fa_fwd_fp8, fa_get_device_status, fa_version)
 
 __all__ = [
     "attention_fwd", "attention_bwd", "decode", "decode_splitkv", "decode_combine", "device_status",
     "fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq", "fa_decode_splitkv", "fa_decode_combine", "fa_decode_num_splits",
     "fa_decode_workspace_bytes", "fa_bwd_workspace_bytes", "fa_decode_chunk", "fa_get_device_status",
-    "FAError",
+    "fp8_quantize_qk", "fp8_quantize_v", "attention_fwd_fp8", "fa_fp8_quantize_qk", "fa_fp8_quantize_v",
+    "fa_fp8_v_workspace_bytes", "fa_fwd_fp8", "FAError",
 ]
 
 
@@ -65,6 +67,50 @@ def attention_fwd(q, k, v, causal: bool = False, scale: float | None = None, out
     fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
            causal, scale, _dt(q), _stream(dev))
     return o, l
+
+
+def fp8_quantize_qk(x, signs=None):
+    """E4M3 codes [B, N, H, d] (uint8) and block scales [B, H, ceil(N/128)] of Q or K, via ``fa_fp8_quantize_qk``.
+
+    ``signs``: optional float32 CUDA tensor of d values +-1 (rotation before quantization).
+    """
+    torch = _torch()
+    dev = _dev(x) if signs is None else _dev(x, signs)
+    B, N, H, d = x.shape
+    x8 = torch.empty(B, N, H, d, device=dev, dtype=torch.uint8)
+    sc = torch.empty(B, H, (N + 127) // 128, device=dev, dtype=torch.float32)
+    fa_fp8_quantize_qk(x.data_ptr(), x8.data_ptr(), sc.data_ptr(), 0 if signs is None else signs.data_ptr(),
+                       B, H, N, d, _dt(x), _stream(dev))
+    return x8, sc
+
+
+def fp8_quantize_v(v):
+    """Transposed E4M3 codes [B, Hkv, d, Nk_pad] and per-head scales [B, Hkv] of V, via ``fa_fp8_quantize_v``."""
+    torch = _torch()
+    dev = _dev(v)
+    B, Nk, H, d = v.shape
+    v8t = torch.empty(B, H, d, (Nk + 15) // 16 * 16, device=dev, dtype=torch.uint8)
+    sc = torch.empty(B, H, device=dev, dtype=torch.float32)
+    ws = torch.empty(fa_fp8_v_workspace_bytes(B, H, Nk), device=dev, dtype=torch.uint8)
+    fa_fp8_quantize_v(v.data_ptr(), v8t.data_ptr(), sc.data_ptr(), ws.data_ptr(), B, H, Nk, d, _dt(v), _stream(dev))
+    return v8t, sc
+
+
+def attention_fwd_fp8(q8, q_scale, k8, k_scale, v8t, v_scale, Nk: int, causal: bool = False,
+                      scale: float | None = None, rotated: bool = False, out_dtype=None):
+    """FP8 forward (``fa_fwd_fp8``) on quantized operands; returns O [B, Nq, Hq, d] and LSE [B, Hq, Nq]."""
+    torch = _torch()
+    dev = _dev(q8, q_scale, k8, k_scale, v8t, v_scale)
+    B, Nq, Hq, d = q8.shape
+    Hkv = k8.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    o = torch.empty(B, Nq, Hq, d, device=dev, dtype=out_dtype)
+    lse = torch.empty(B, Hq, Nq, device=dev, dtype=torch.float32)
+    fa_fwd_fp8(q8.data_ptr(), q_scale.data_ptr(), k8.data_ptr(), k_scale.data_ptr(), v8t.data_ptr(),
+               v_scale.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, causal, scale, rotated,
+               _dt(o), _stream(dev))
+    return o, lse
 
 
 def attention_bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, workspace=None,

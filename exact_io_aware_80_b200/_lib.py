@@ -39,6 +39,10 @@ SIGNATURES = {
     "fa_decode_combine": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "fa_decode_chunk": (_I, [_I, _I]),
     "fa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "fa_fp8_quantize_qk": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "fa_fp8_v_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I]),
+    "fa_fp8_quantize_v": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "fa_get_device_status": (_I, [_P]),
     "fa_watchdog_selftest": (_I, [_I, _P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
@@ -129,6 +133,24 @@ def fa_decode_splitkv(q, k_cache, v_cache, seqlens_k, B, Hq, Hkv, Nk_max, d, sca
 def fa_decode_combine(workspace, o, lse, seqlens_k, B, Hq, num_splits, d, dt, stream):
     return _check("fa_decode_combine", load().fa_decode_combine(workspace, o, lse, seqlens_k, B, Hq, num_splits, d,
                                                                 dt, stream))
+
+
+def fa_fp8_quantize_qk(x, x8, scales, signs, B, H, N, d, dt, stream):
+    return _check("fa_fp8_quantize_qk", load().fa_fp8_quantize_qk(x, x8, scales, signs, B, H, N, d, dt, stream))
+
+
+def fa_fp8_v_workspace_bytes(B, Hkv, Nk):
+    return load().fa_fp8_v_workspace_bytes(B, Hkv, Nk)
+
+
+def fa_fp8_quantize_v(v, v8t, scale, workspace, B, Hkv, Nk, d, dt, stream):
+    return _check("fa_fp8_quantize_v", load().fa_fp8_quantize_v(v, v8t, scale, workspace, B, Hkv, Nk, d, dt, stream))
+
+
+def fa_fwd_fp8(q8, q_scale, k8, k_scale, v8t, v_scale, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, rotated, dt,
+               stream):
+    return _check("fa_fwd_fp8", load().fa_fwd_fp8(q8, q_scale, k8, k_scale, v8t, v_scale, o, lse, B, Hq, Hkv, Nq, Nk,
+                                                  d, int(causal), scale, int(rotated), dt, stream))
 
 
 def fa_watchdog_selftest(limit_us, stream):

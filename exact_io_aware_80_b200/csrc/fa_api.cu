@@ -81,6 +81,48 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   return from_cuda(fa::launch_fwd_sm100(a, s));
 }
 
+fa_status fa_fp8_quantize_qk(const void* x, void* x8, float* scales, const float* signs, int B, int H, int N, int d,
+                             fa_dtype dt, fa_stream_t stream) {
+  if (!x || !x8 || !scales) return FA_ERR_INVALID;
+  fa_status st = check_shape(B, H, H, N, N, d, 0, dt);
+  if (st != FA_OK) return st;
+  if (!aligned16(x) || !aligned16(x8) || !aligned4(scales) || (signs && !aligned4(signs))) return FA_ERR_ALIGN;
+  fa::Fp8QuantArgs a{x, x8, scales, signs, nullptr, B, H, N, d, dt == FA_BF16 ? 1 : 0};
+  return from_cuda(fa::launch_fp8_quant_qk(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t fa_fp8_v_workspace_bytes(int B, int Hkv, int Nk) {
+  if (B < 1 || Hkv < 1 || Nk < 1) return 0;
+  return (size_t)B * Hkv * ((Nk + 127) / 128) * sizeof(float);
+}
+
+fa_status fa_fp8_quantize_v(const void* v, void* v8t, float* scale, void* workspace, int B, int Hkv, int Nk, int d,
+                            fa_dtype dt, fa_stream_t stream) {
+  if (!v || !v8t || !scale || !workspace) return FA_ERR_INVALID;
+  fa_status st = check_shape(B, Hkv, Hkv, Nk, Nk, d, 0, dt);
+  if (st != FA_OK) return st;
+  if (!aligned16(v) || !aligned16(v8t) || !aligned16(workspace) || !aligned4(scale)) return FA_ERR_ALIGN;
+  fa::Fp8QuantArgs a{v, v8t, scale, nullptr, static_cast<float*>(workspace), B, Hkv, Nk, d, dt == FA_BF16 ? 1 : 0};
+  return from_cuda(fa::launch_fp8_quant_v(a, static_cast<cudaStream_t>(stream)));
+}
+
+fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const float* k_scale, const void* v8t,
+                     const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                     int causal, float scale, int rotated, fa_dtype out_dt, fa_stream_t stream) {
+  if (!q8 || !q_scale || !k8 || !k_scale || !v8t || !v_scale || !o || !lse) return FA_ERR_INVALID;
+  fa_status st = check_shape(B, Hq, Hkv, Nq, Nk, d, causal, out_dt);
+  if (st != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8t) || !aligned16(o) || !aligned4(lse) || !aligned4(q_scale) ||
+      !aligned4(k_scale) || !aligned4(v_scale))
+    return FA_ERR_ALIGN;
+  if (!fa::tma_available()) return FA_ERR_CUDA;
+  fa::Fp8AttnArgs a{q8,  q_scale, k8, k_scale, v8t, v_scale, o, lse, B, Hq, Hkv, Nq, Nk, d, causal ? 1 : 0, scale,
+                    rotated ? 1 : 0, out_dt == FA_BF16 ? 1 : 0, status_ptr()};
+  if (!a.status) return FA_ERR_CUDA;
+  return from_cuda(fa::launch_fwd_fp8_sm100(a, static_cast<cudaStream_t>(stream)));
+}
+
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq) {
   if (B < 1 || Hq < 1 || Nq < 1) return 0;
   return (size_t)B * Hq * Nq * sizeof(float);

@@ -30,6 +30,13 @@
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // Causal tiles beyond the diagonal are skipped; the diagonal and ragged
 // tail tiles are masked per row.
+//
+// The same kernel, instantiated with F8, is the FP8 forward pass (FA-3's
+// low-precision variant; see fp8_quant.cu for the operand formats): Q, K and
+// the transposed V arrive as E4M3 codes, the MMAs run as kind::f8f6f4 (K = 32
+// per instruction), every block's scores are scaled by the Q and K block
+// scales, P is rounded to E4M3 for the P V product, and the epilogue applies
+// V's scale.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -62,15 +69,17 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when m grows
 __host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }        // S_t / P_t
 __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * t; }  // O_t
 
-template <int D>
+template <int D, bool F8>
 struct Smem {
-  static constexpr int kPanel = 128 * 128;  // one [128 rows][64 cols] 16-bit panel, bytes
-  static constexpr int kTile = (D / 64) * kPanel;
+  static constexpr int kPanel = 128 * 128;  // one [128 rows][128 bytes] swizzled panel
+  // a Q, K or V tile: 16-bit [128][D] as D / 64 panels, or E4M3 [128][D = 128] as one panel
+  static constexpr int kTile = F8 ? 128 * D : (D / 64) * kPanel;
+  static constexpr int kTileOut = (D / 64) * kPanel;  // a 16-bit O tile
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kTiles * kTile;
   static constexpr int kOffV = kOffK + kStages * kTile;
   static constexpr int kOffStage = kOffV + kStages * kTile;  // one 16-bit O tile on its way to a TMA store
-  static constexpr int kOffBar = kOffStage + kTile;
+  static constexpr int kOffBar = kOffStage + kTileOut;
   // kBarQ/kBarQEmpty: the query tiles of a work tile landed / may be replaced; kBarO + t: tile t's
   // last PV finished; kBarOFree + t: the epilogue of tile t has read O_t from TMEM;
   // kBarStageFull + t: tile t's rows are in the stage buffer; kBarStageDone + t: the TMA store of
@@ -91,6 +100,11 @@ struct Params {
   int* status;
   int num_mblk;  // 256-row blocks per (b, h)
   int num_work;  // num_mblk * Hq * B work tiles
+  // FP8 only: Q / K scales per 128-row block ([B,Hq,nqb], [B,Hkv,nkb]), V scale per head [B,Hkv]
+  const float* q_scale;
+  const float* k_scale;
+  const float* v_scale;
+  int nqb, nkb;
 };
 
 // Work tile w of the persistent schedule: row block, query head, batch.  Causal
@@ -116,11 +130,11 @@ __device__ __forceinline__ Work work_at(const Params& p, int w) {
   return x;
 }
 
-template <typename T, int D, bool CAUSAL>
+template <typename T, int D, bool CAUSAL, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, Params p) {
-  using L = Smem<D>;
+  using L = Smem<D, F8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
@@ -178,11 +192,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (wl > 0 && !mbar_wait(bar(L::kBarQEmpty), (wl - 1) & 1, abort_flag, p.status)) break;
         mbar_expect_tx(bar(L::kBarQ), kTiles * L::kTile);
 #pragma unroll
-        for (int t = 0; t < kTiles; ++t)
+        for (int t = 0; t < kTiles; ++t) {
+          if constexpr (F8) {
+            tma_load_4d(sb + L::kOffQ + t * L::kTile, &tmQ, bar(L::kBarQ), 0, x.hq, m0 + t * kBM, x.b);
+          } else {
 #pragma unroll
-          for (int pn = 0; pn < D / 64; ++pn)
-            tma_load_4d(sb + L::kOffQ + t * L::kTile + pn * L::kPanel, &tmQ, bar(L::kBarQ), 64 * pn, x.hq,
-                        m0 + t * kBM, x.b);
+            for (int pn = 0; pn < D / 64; ++pn)
+              tma_load_4d(sb + L::kOffQ + t * L::kTile + pn * L::kPanel, &tmQ, bar(L::kBarQ), 64 * pn, x.hq,
+                          m0 + t * kBM, x.b);
+          }
+        }
         last_q = wl;
         bool stop = false;
         for (int j = 0; j < nblk; ++j, ++g) {
@@ -192,20 +211,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_expect_tx(bar(L::kBarKFull + st), L::kTile);
+          if constexpr (F8) {
+            tma_load_4d(sb + L::kOffK + st * L::kTile, &tmK, bar(L::kBarKFull + st), 0, hk, j * kBN, x.b);
+          } else {
 #pragma unroll
-          for (int pn = 0; pn < D / 64; ++pn)
-            tma_load_4d(sb + L::kOffK + st * L::kTile + pn * L::kPanel, &tmK, bar(L::kBarKFull + st), 64 * pn, hk,
-                        j * kBN, x.b);
+            for (int pn = 0; pn < D / 64; ++pn)
+              tma_load_4d(sb + L::kOffK + st * L::kTile + pn * L::kPanel, &tmK, bar(L::kBarKFull + st), 64 * pn, hk,
+                          j * kBN, x.b);
+          }
           if (u > 0 && !mbar_wait(bar(L::kBarVEmpty + st), (u - 1) & 1, abort_flag, p.status)) {
             last_u[st] = u;  // K of this use is in flight
             stop = true;
             break;
           }
           mbar_expect_tx(bar(L::kBarVFull + st), L::kTile);
+          if constexpr (F8) {
+            // V transposed: [d rows][128 keys], keys innermost
+            tma_load_4d(sb + L::kOffV + st * L::kTile, &tmV, bar(L::kBarVFull + st), j * kBN, 0, hk, x.b);
+          } else {
 #pragma unroll
-          for (int pn = 0; pn < D / 64; ++pn)
-            tma_load_4d(sb + L::kOffV + st * L::kTile + pn * L::kPanel, &tmV, bar(L::kBarVFull + st), 64 * pn, hk,
-                        j * kBN, x.b);
+            for (int pn = 0; pn < D / 64; ++pn)
+              tma_load_4d(sb + L::kOffV + st * L::kTile + pn * L::kPanel, &tmV, bar(L::kBarVFull + st), 64 * pn, hk,
+                          j * kBN, x.b);
+          }
           last_u[st] = u;
         }
         if (stop) break;
@@ -224,23 +252,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr bool kBf16 = Elem<T>::kBf16;
-      constexpr uint32_t idq = idesc_f16(kBf16, kBM, kBN, false);
-      constexpr uint32_t idv = idesc_f16(kBf16, kBM, D, true);
+      constexpr uint32_t idq = F8 ? idesc_e4m3(kBM, kBN) : idesc_f16(kBf16, kBM, kBN, false);
+      constexpr uint32_t idv = F8 ? idesc_e4m3(kBM, D) : idesc_f16(kBf16, kBM, D, true);
       auto qk = [&](int t, int st) {
+        if constexpr (F8) {
+          // 32 E4M3 values of d = 32 bytes per step along the 128-byte rows
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2) * L::kPanel + (kk & 3) * 32;
-          const uint64_t a = sdesc_sw128(sb + L::kOffQ + t * L::kTile + ko, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sb + L::kOffK + st * L::kTile + ko, 16, 1024);
-          mma_ss(tbase + col_s(t), a, bd, idq, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 32; ++kk) {
+            const uint64_t a = sdesc_sw128(sb + L::kOffQ + t * L::kTile + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sb + L::kOffK + st * L::kTile + kk * 32, 16, 1024);
+            mma_ss_f8(tbase + col_s(t), a, bd, idq, kk > 0 ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t ko = (kk >> 2) * L::kPanel + (kk & 3) * 32;
+            const uint64_t a = sdesc_sw128(sb + L::kOffQ + t * L::kTile + ko, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sb + L::kOffK + st * L::kTile + ko, 16, 1024);
+            mma_ss(tbase + col_s(t), a, bd, idq, kk > 0 ? 1u : 0u);
+          }
         }
       };
       auto pv = [&](int t, int st, bool first) {
+        if constexpr (F8) {
+          // P: 4 E4M3 codes per TMEM column (32 keys = 8 columns per step); V^T K-major
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          // V stored [keys][d]: B is N(=d)-major; 16 keys = two 8-row groups of 128 B
-          const uint64_t bd = sdesc_sw128(sb + L::kOffV + st * L::kTile + kk * 2048, L::kPanel, 1024);
-          mma_ts(tbase + col_o(t), tbase + col_s(t) + kk * 8, bd, idv, (!first || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kBN / 32; ++kk) {
+            const uint64_t bd = sdesc_sw128(sb + L::kOffV + st * L::kTile + kk * 32, 16, 1024);
+            mma_ts_f8(tbase + col_o(t), tbase + col_s(t) + kk * 8, bd, idv, (!first || kk > 0) ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            // V stored [keys][d]: B is N(=d)-major; 16 keys = two 8-row groups of 128 B
+            const uint64_t bd = sdesc_sw128(sb + L::kOffV + st * L::kTile + kk * 2048, L::kPanel, 1024);
+            mma_ts(tbase + col_o(t), tbase + col_s(t) + kk * 8, bd, idv, (!first || kk > 0) ? 1u : 0u);
+          }
         }
       };
       bool ok = true;
@@ -315,6 +362,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nblk = blocks_of(x.mblk);
       const int row_first = m0 + t * kBM;
       const int row = row_first + wq * 32 + lane;
+      const int hk = h / (p.Hq / p.Hkv);
+      float cq = c;  // FP8: times the Q tile's block scale
+      if constexpr (F8) cq = c * p.q_scale[((long)b * p.Hq + h) * p.nqb + min(row_first / kBM, p.nqb - 1)];
       float m_ref = -INFINITY, l = 0.f;
         for (int j = 0; j < nblk; ++j, ++g) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + t), g & 1, abort_flag, p.status));
@@ -340,6 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             s[96 + i] = __uint_as_float(r3[i]);
           }
         }
+        float cj = cq;  // FP8: times the K block's scale
+        if constexpr (F8) cj = cq * p.k_scale[((long)b * p.Hkv + hk) * p.nkb + j];
         const int kbase = j * kBN;
         if (kbase + kBN > p.Nk || (CAUSAL && kbase + kBN - 1 > row_first + off)) {
           int lim = p.Nk - kbase;
@@ -356,13 +408,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           mx[2] = max3(mx[2], s[i + 4], s[i + 5]);
           mx[3] = max3(mx[3], s[i + 6], s[i + 7]);
         }
-        const float mxs = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
+        const float mxs = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * cj;
         const bool resc = mxs > m_ref + kRescaleThreshold;
         const float corr = resc ? ex2(m_ref - mxs) : 1.f;
         if (resc) m_ref = mxs;
         l *= corr;
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-        const float2 c2 = make_float2(c, c), nm2 = make_float2(-mu, -mu);
+        const float2 c2 = make_float2(cj, cj), nm2 = make_float2(-mu, -mu);
         float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -374,10 +426,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float2 bb = exp2_pair(__ffma2_rn(make_float2(s[c0 + 2], s[c0 + 3]), c2, nm2), 32 * half + i + 1);
             rs0 = __fadd2_rn(rs0, a);
             rs1 = __fadd2_rn(rs1, bb);
-            pk[i] = Elem<T>::pack(a.x, a.y);
-            pk[i + 1] = Elem<T>::pack(bb.x, bb.y);
+            if constexpr (F8) {
+              pk[i >> 1] = pack_e4m3x4(a.x, a.y, bb.x, bb.y);  // keys c0 .. c0 + 3 in one column
+            } else {
+              pk[i] = Elem<T>::pack(a.x, a.y);
+              pk[i + 1] = Elem<T>::pack(bb.x, bb.y);
+            }
           }
-          tmem_st32(tS + 32 * half, pk);
+          if constexpr (F8) {
+            tmem_st16(tS + 16 * half, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+          } else {
+            tmem_st32(tS + 32 * half, pk);
+          }
         }
         l += (rs0.x + rs0.y) + (rs1.x + rs1.y);
         if (__any_sync(0xffffffffu, resc && j > 0)) {
@@ -417,7 +477,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         // O / l as 16-bit into the stage buffer, laid out as the TMA box expects: 64-column
         // panels of 128-byte rows, 16-byte chunk c of row r at chunk c ^ (r & 7)
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        float num = 1.f;  // FP8: V's scale
+        if constexpr (F8) num = p.v_scale[(long)b * p.Hkv + hk];
+        const float inv = l > 0.f ? num / l : 0.f;
         const int rr = wq * 32 + lane;
         const uint32_t srow = sb + L::kOffStage + rr * 128;
         auto o2 = [&](int i) { return Elem<T>::pack(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv); };
@@ -469,12 +531,45 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   const int num_mblk = (a.Nq + kTiles * kBM - 1) / (kTiles * kBM);
   const long long num_work = (long long)num_mblk * a.Hq * a.B;
   if (num_work > (1ll << 31) - 1) return cudaErrorInvalidValue;
-  Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, a.scale * kLog2e, a.status, num_mblk, (int)num_work};
-  auto kern = fwd_sm100_kernel<T, D, CAUSAL>;
-  const int smem = Smem<D>::kBytes;
+  Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, a.scale * kLog2e, a.status, num_mblk, (int)num_work,
+           nullptr, nullptr, nullptr, 0, 0};
+  auto kern = fwd_sm100_kernel<T, D, CAUSAL, false>;
+  const int smem = Smem<D, false>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   // persistent: one CTA per SM (the shared-memory footprint allows no more), looping over work tiles
+  const int grid = (int)std::min<long long>(num_work, device_sm_count());
+  kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mo, p);
+  return cudaGetLastError();
+}
+
+// FP8: d = 128.  Q/K maps over E4M3 [B][N][H][128] (box 128 bytes x 1 x 128 rows x 1),
+// V map over the transposed codes [B][Hkv][128][Nk_pad] (box 128 keys x 128 rows x 1 x 1).
+template <typename T, bool CAUSAL>
+cudaError_t launch_f8(const Fp8AttnArgs& a, cudaStream_t s) {
+  constexpr int D = 128;
+  const uint64_t npad = (uint64_t)(a.Nk + 15) / 16 * 16;
+  const uint64_t dq[4] = {D, (uint64_t)a.Hq, (uint64_t)a.Nq, (uint64_t)a.B};
+  const uint64_t sq[3] = {D, (uint64_t)a.Hq * D, (uint64_t)a.Nq * a.Hq * D};
+  const uint64_t dk[4] = {D, (uint64_t)a.Hkv, (uint64_t)a.Nk, (uint64_t)a.B};
+  const uint64_t sk[3] = {D, (uint64_t)a.Hkv * D, (uint64_t)a.Nk * a.Hkv * D};
+  const uint64_t dv[4] = {npad, D, (uint64_t)a.Hkv, (uint64_t)a.B};
+  const uint64_t sv[3] = {npad, D * npad, (uint64_t)a.Hkv * D * npad};
+  const uint32_t box_qk[4] = {128, 1, kBM, 1}, box_v[4] = {kBN, D, 1, 1};
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map_u8(&mq, a.q8, dq, sq, box_qk) || !make_map_u8(&mk, a.k8, dk, sk, box_qk) ||
+      !make_map_u8(&mv, a.v8t, dv, sv, box_v) || !make_map(&mo, a.o, Elem<T>::kBf16, D, a.Hq, a.Nq, a.B, kBM))
+    return cudaErrorInvalidValue;
+  const int num_mblk = (a.Nq + kTiles * kBM - 1) / (kTiles * kBM);
+  const long long num_work = (long long)num_mblk * a.Hq * a.B;
+  if (num_work > (1ll << 31) - 1) return cudaErrorInvalidValue;
+  const float sl2 = a.scale * kLog2e / (a.rotated ? (float)D : 1.f);
+  Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, sl2, a.status, num_mblk, (int)num_work,
+           a.q_scale, a.k_scale, a.v_scale, (a.Nq + kBM - 1) / kBM, (a.Nk + kBN - 1) / kBN};
+  auto kern = fwd_sm100_kernel<T, D, CAUSAL, true>;
+  const int smem = Smem<D, true>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
   const int grid = (int)std::min<long long>(num_work, device_sm_count());
   kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mo, p);
   return cudaGetLastError();
@@ -494,6 +589,11 @@ bool fwd_sm100_supported(const AttnArgs& a) {
 
 cudaError_t launch_fwd_sm100(const AttnArgs& a, cudaStream_t s) {
   return a.bf16 ? launch_t<__nv_bfloat16>(a, s) : launch_t<__half>(a, s);
+}
+
+cudaError_t launch_fwd_fp8_sm100(const Fp8AttnArgs& a, cudaStream_t s) {
+  if (a.bf16) return a.causal ? launch_f8<__nv_bfloat16, true>(a, s) : launch_f8<__nv_bfloat16, false>(a, s);
+  return a.causal ? launch_f8<__half, true>(a, s) : launch_f8<__half, false>(a, s);
 }
 
 }  // namespace fa

@@ -63,6 +63,39 @@ struct CombineArgs {
   int bf16;
 };
 
+// FP8 operand preparation (fp8_quant.cu).  Q/K: x [B,N,H,d] 16-bit -> x8 codes [B,N,H,d],
+// scales [B,H,ceil(N/128)], optional rotation signs [d].  V: x [B,N,H,d] -> x8 codes
+// [B,H,d,Npad] (Npad = N rounded up to 16), scales [B,H], work = per-block amax
+// [B,H,ceil(N/128)] fp32.
+struct Fp8QuantArgs {
+  const void* x;
+  void* x8;
+  float* scales;
+  const float* signs;
+  float* work;
+  int B, H, N, d;
+  int bf16;
+};
+
+// FP8 forward: E4M3 Q/K codes [B,N,H,d] with block scales, V codes transposed
+// [B,Hkv,d,Nk_pad] with one scale per head; O in the 16-bit type `bf16` names.
+struct Fp8AttnArgs {
+  const void* q8;
+  const float* q_scale;
+  const void* k8;
+  const float* k_scale;
+  const void* v8t;
+  const float* v_scale;
+  void* o;
+  float* lse;
+  int B, Hq, Hkv, Nq, Nk, d;
+  int causal;
+  float scale;  // softmax scale of the original scores
+  int rotated;  // Q and K were rotated: the scores are d times the original ones
+  int bf16;
+  int* status;
+};
+
 // TMA descriptors (tma.cu).  make_map: 4-D map over a BSHD tensor [B][N][H][D]
 // (innermost d, then head, row, batch); box = 64 columns (128 bytes, 128-byte
 // swizzle) x 1 head x `rows` rows x 1 batch.  Out-of-range rows read as zero.
@@ -70,10 +103,19 @@ bool tma_available();
 // Streaming multiprocessors of the current device (148 if the query fails).
 int device_sm_count();
 bool make_map(CUtensorMap* m, const void* base, bool bf16, int D, int H, int N, int B, int rows);
+// 4-D map over bytes: dims (innermost first), strides of dims 1..3 in bytes, box,
+// 128-byte swizzle (the box's innermost extent must be 128 bytes).
+bool make_map_u8(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides[3],
+                 const uint32_t box[4]);
 
 // Forward on tcgen05 / TMEM / TMA (warp-specialised), d = 128 and 64.
 cudaError_t launch_fwd_sm100(const AttnArgs& a, cudaStream_t s);
 bool fwd_sm100_supported(const AttnArgs& a);
+
+// FP8 forward on tcgen05 kind::f8f6f4, d = 128 (fwd_sm100.cu).
+cudaError_t launch_fwd_fp8_sm100(const Fp8AttnArgs& a, cudaStream_t s);
+cudaError_t launch_fp8_quant_qk(const Fp8QuantArgs& a, cudaStream_t s);
+cudaError_t launch_fp8_quant_v(const Fp8QuantArgs& a, cudaStream_t s);
 
 cudaError_t launch_bwd_preprocess(const BwdArgs& a, cudaStream_t s);
 // Backward dK/dV and dQ on tcgen05 / TMEM / TMA, d = 128 and 64.

@@ -184,6 +184,60 @@ fa_status fa_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
                             void* o, float* lse, int B, int Hq, int Hkv, int Nk_max, int d, float scale,
                             int num_splits, fa_dtype dt, fa_stream_t stream);
 
+/* ------------------------------------------------------------------------------
+ * FP8 forward pass ("FlashAttention-2 (KO)", FA-3 paragraph: low-precision FP8
+ * with incoherent processing; smithlab guide, version table: FP8 is forward
+ * only).  The pages give no formats; the library fixes them:
+ *  - codes are E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits,
+ *    largest finite 448), converted with round-to-nearest-even and saturation;
+ *  - Q and K: one fp32 scale per (batch, head, 128-row block), s = amax / 448
+ *    (1 for an all-zero block), code = E4M3(y / s) with a correctly rounded
+ *    fp32 division;
+ *  - incoherent processing (optional): before quantization the rows of Q and
+ *    K are multiplied by `signs` (d values, each +1 or -1) and then by the
+ *    unnormalised d x d Walsh-Hadamard matrix, in fp32 with the butterflies
+ *    (a, b) -> (a + b, a - b) taken for h = 1, 2, 4, ..., d / 2; the scores
+ *    become d times the original ones, which fa_fwd_fp8 undoes when `rotated`;
+ *  - V: one fp32 scale per (batch, kv head) over all Nk keys, codes stored
+ *    transposed as [B, Hkv, d, Nk_pad], Nk_pad = Nk rounded up to 16, zero
+ *    codes in the padding.
+ * d must be 128 for fa_fwd_fp8 (64 or 128 for the quantizers).
+ * ---------------------------------------------------------------------------- */
+
+/*
+ * Quantize Q or K.  x: [B, N, H, d] 16-bit (dt); x8: [B, N, H, d] bytes;
+ * scales: [B, H, ceil(N / 128)] fp32; signs: d fp32 values of +-1 on the device,
+ * or NULL for no rotation.  x, x8 16-byte aligned, scales and signs 4-byte
+ * aligned.  Writes every code and scale; FA_ERR_INVALID / _UNSUPPORTED /
+ * _ALIGN on bad arguments, FA_ERR_CUDA if the launch fails.
+ */
+fa_status fa_fp8_quantize_qk(const void* x, void* x8, float* scales, const float* signs, int B, int H, int N, int d,
+                             fa_dtype dt, fa_stream_t stream);
+
+/* Workspace bytes of fa_fp8_quantize_v: B * Hkv * ceil(Nk / 128) fp32 block maxima (0 on bad sizes). */
+size_t fa_fp8_v_workspace_bytes(int B, int Hkv, int Nk);
+
+/*
+ * Quantize V.  v: [B, Nk, Hkv, d] 16-bit; v8t: [B, Hkv, d, Nk_pad] bytes
+ * (Nk_pad = Nk rounded up to 16); scale: [B, Hkv] fp32; workspace as sized by
+ * fa_fp8_v_workspace_bytes.  v, v8t, workspace 16-byte aligned, scale 4-byte.
+ */
+fa_status fa_fp8_quantize_v(const void* v, void* v8t, float* scale, void* workspace, int B, int Hkv, int Nk,
+                            int d, fa_dtype dt, fa_stream_t stream);
+
+/*
+ * FP8 forward.  q8 [B, Nq, Hq, 128] and k8 [B, Nk, Hkv, 128] E4M3 codes with
+ * scales [B, Hq, ceil(Nq / 128)] and [B, Hkv, ceil(Nk / 128)]; v8t [B, Hkv,
+ * 128, Nk_pad] with scale [B, Hkv] (as written by the quantizers above).
+ * Computes S = scale * (Q K^T) (divided by d when `rotated`), the online
+ * softmax of the 16-bit path with P rounded to E4M3 for the P V product, and
+ * writes o [B, Nq, Hq, 128] in `out_dt` and lse [B, Hq, Nq] fp32 (natural log
+ * of the scaled scores).  Same causal, GQA, alignment and error rules as fa_fwd.
+ */
+fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const float* k_scale, const void* v8t,
+                     const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                     int causal, float scale, int rotated, fa_dtype out_dt, fa_stream_t stream);
+
 /*
  * Synchronises `stream`, then reads and clears the device status word that the
  * kernels set when a bounded wait runs out (FA_ERR_TIMEOUT) or a device-side

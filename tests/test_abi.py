@@ -126,3 +126,30 @@ def test_binding_without_gpu_fails_loudly():
     q = torch.zeros(1, 8, 2, 64, dtype=torch.float16)
     with pytest.raises(ValueError):
         fa.attention_fwd(q, q, q)
+
+
+def test_fp8_entry_points_reject_bad_arguments(lib):
+    from exact_io_aware_80_b200 import _lib
+    assert _lib.fa_fp8_v_workspace_bytes(2, 8, 300) == 2 * 8 * 3 * 4
+    assert _lib.fa_fp8_v_workspace_bytes(0, 8, 300) == 0
+    # x, x8, scales, signs, B, H, N, d, dt, stream
+    assert lib.fa_fp8_quantize_qk(0, FAKE, FAKE, 0, 1, 2, 8, 128, 1, None) == -1
+    assert lib.fa_fp8_quantize_qk(FAKE, FAKE, FAKE, 0, 1, 2, 8, 96, 1, None) == -2
+    assert lib.fa_fp8_quantize_qk(FAKE + 8, FAKE, FAKE, 0, 1, 2, 8, 128, 1, None) == -3
+    assert lib.fa_fp8_quantize_qk(FAKE, FAKE, FAKE, FAKE + 2, 1, 2, 8, 128, 1, None) == -3
+    assert lib.fa_fp8_quantize_v(FAKE, FAKE, FAKE, 0, 1, 2, 8, 128, 1, None) == -1
+    assert lib.fa_fp8_quantize_v(FAKE, FAKE, FAKE, FAKE, 1, 2, 0, 128, 1, None) == -1
+    # q8, qs, k8, ks, v8t, vs, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, rotated, dt, stream
+    base = [FAKE] * 8 + [1, 4, 2, 8, 8, 128, 0, 0.1, 0, 1, None]
+    bad = list(base)
+    bad[13] = 64  # the FP8 forward takes d = 128 only
+    assert lib.fa_fwd_fp8(*bad) == -2
+    bad = list(base)
+    bad[9] = 5  # Hq % Hkv
+    assert lib.fa_fwd_fp8(*bad) == -1
+    bad = list(base)
+    bad[1] = 0  # q_scale
+    assert lib.fa_fwd_fp8(*bad) == -1
+    bad = list(base)
+    bad[4] = FAKE + 4  # v8t misaligned
+    assert lib.fa_fwd_fp8(*bad) == -3

@@ -18,7 +18,8 @@ import math
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "get", "make_inputs", "make_decode_inputs", "seqlens_for", "workload_inputs"]
+__all__ = ["Workload", "WORKLOADS", "get", "make_inputs", "make_decode_inputs", "seqlens_for", "workload_inputs",
+           "rotation_signs"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -75,6 +76,13 @@ def make_inputs(B, Hq, Hkv, Nq, Nk, d, dtype=torch.bfloat16, seed_base=0, with_d
         return q, k, v
     do = _normal((B, Nq, Hq, d), seed_base + 3, dtype, device)
     return q, k, v, do
+
+
+def rotation_signs(d: int, seed: int, device="cpu") -> torch.Tensor:
+    """fp32 [d] of +-1, each sign drawn with probability 1/2 by a generator seeded ``seed``."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    bits = torch.randint(0, 2, (d,), generator=g)
+    return (bits.float() * 2 - 1).to(device)
 
 
 def seqlens_for(B: int, Nk_max: int, seed: int, lo: int = 1024) -> torch.Tensor:
