@@ -270,6 +270,8 @@ def run_ours(args):
 
     decode = None if args.no_decode else run_decode(args, torch, fa, _lib, workloads, dev, stream, world, peaks,
                                                     peaks_kind)
+    fp8 = None if args.no_fp8 else run_fp8(args, torch, fa, _lib, workloads, w, q, k, v, dev, stream, world, peaks,
+                                           peaks_kind)
     e2e = run_e2e(args, torch, fa, w, q, k, v, do, dev, stream, world, F) if not args.no_e2e else None
 
     cpu = None
@@ -293,6 +295,7 @@ def run_ours(args):
                   "bwd_frac_of_measured": round(bwd_tflops / peak, 4),
                   "per_kernel_ms": {kk: round(vv, 4) for kk, vv in per.items()}},
         "decode": decode,
+        "fp8": fp8,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -367,6 +370,69 @@ def run_decode(args, torch, fa, _lib, workloads, dev, stream, world, peaks, peak
                          "traffic": traffic_for("decode_split_kernel"), "peak_source": f"{peaks_kind} hbm_gbs",
                          "algorithmic_bytes_per_launch": split_bytes},
             "gpu_launches": 2 * K}
+
+
+def run_fp8(args, torch, fa, _lib, workloads, w, q, k, v, dev, stream, world, peaks, peaks_kind):
+    """FP8 forward on the same GQA inputs: E4M3 quantization (Q, K rotated) + the fp8 forward kernel."""
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.Nq, w.d
+    sh = stream.cuda_stream
+    signs = workloads.rotation_signs(d, 1000 * w.id + 9, device=dev)
+    nb = (N + 127) // 128
+    npad = (N + 15) // 16 * 16
+    q8 = torch.empty(B, N, Hq, d, device=dev, dtype=torch.uint8)
+    k8 = torch.empty(B, N, Hkv, d, device=dev, dtype=torch.uint8)
+    v8t = torch.empty(B, Hkv, d, npad, device=dev, dtype=torch.uint8)
+    qs = torch.empty(B, Hq, nb, device=dev, dtype=torch.float32)
+    ks = torch.empty(B, Hkv, nb, device=dev, dtype=torch.float32)
+    vs = torch.empty(B, Hkv, device=dev, dtype=torch.float32)
+    vws = torch.empty(fa.fa_fp8_v_workspace_bytes(B, Hkv, N), device=dev, dtype=torch.uint8)
+    o = torch.empty(B, N, Hq, d, device=dev, dtype=torch.bfloat16)
+    lse = torch.empty(B, Hq, N, device=dev, dtype=torch.float32)
+    dt = _lib.FA_BF16
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        _lib.fa_fp8_quantize_qk(q.data_ptr(), q8.data_ptr(), qs.data_ptr(), signs.data_ptr(), B, Hq, N, d, dt, sh)
+        _lib.fa_fp8_quantize_qk(k.data_ptr(), k8.data_ptr(), ks.data_ptr(), signs.data_ptr(), B, Hkv, N, d, dt, sh)
+        _lib.fa_fp8_quantize_v(v.data_ptr(), v8t.data_ptr(), vs.data_ptr(), vws.data_ptr(), B, Hkv, N, d, dt, sh)
+        if ev:
+            ev[1].record(stream)
+        _lib.fa_fwd_fp8(q8.data_ptr(), qs.data_ptr(), k8.data_ptr(), ks.data_ptr(), v8t.data_ptr(), vs.data_ptr(),
+                        o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, N, d, 1, w.scale, 1, dt, sh)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    barrier(torch, world)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(torch, world)
+    ms = max_over_ranks(torch, world, t0.elapsed_time(t1)) / K
+    if fa.device_status() != 0:
+        raise RuntimeError("kernel status word set during the fp8 section")
+    quant_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in evs)
+    fwd_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in evs)
+    F = attn_flops(B, Hq, N, N, d, True)
+    key = "bf16_tflops_sustained" if ms * K >= 2000 else "bf16_tflops"
+    peak = 2.0 * float(peaks.get(key, FALLBACK_PEAKS[key]))  # e4m3 dense rate = 2x bf16 (nominal ratio)
+    ach = F / (fwd_ms * 1e-3) / 1e12
+    return {"workload": f"FP8 (E4M3) forward, Q/K rotated: B={B} Hq={Hq} Hkv={Hkv} N={N} d={d} causal, bf16 in/out",
+            "ms_per_step": round(ms, 4), "quantize_ms": round(quant_ms, 4), "fwd_ms": round(fwd_ms, 4),
+            "fwd_tflops": round(ach, 1), "value": round(world * F / (ms * 1e-3) / 1e12, 1), "unit": "TFLOP/s",
+            "roofline": {"bound": "tensor", "kernel": "fwd_sm100_kernel (F8)", "achieved": round(ach, 1),
+                         "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                         "peak_source": f"{peaks_kind} {key} x 2 (nominal e4m3 / bf16 ratio)",
+                         "algorithmic_flops_per_launch": F},
+            "gpu_launches": 5 * K}
 
 
 def run_e2e(args, torch, fa, w, q, k, v, do, dev, stream, world, F):
@@ -496,6 +562,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode section (profiling runs)")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 forward section (profiling runs)")
     ap.add_argument("--decode-b", type=int, default=0,
                     help="override B of the decode workload (profiling runs on a smaller case)")
     ap.add_argument("--seq", type=int, default=0,
