@@ -19,7 +19,7 @@ import math
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "get", "make_inputs", "make_decode_inputs", "seqlens_for", "workload_inputs",
-           "rotation_signs"]
+           "rotation_signs", "block_mask_local", "block_mask_random"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -83,6 +83,20 @@ def rotation_signs(d: int, seed: int, device="cpu") -> torch.Tensor:
     g = torch.Generator(device="cpu").manual_seed(seed)
     bits = torch.randint(0, 2, (d,), generator=g)
     return (bits.float() * 2 - 1).to(device)
+
+
+def block_mask_local(B: int, Hq: int, nqb: int, nkb: int, window: int, sink: int = 1) -> torch.Tensor:
+    """uint8 [B, Hq, nqb, nkb]: query block I sees key blocks I - window + 1 .. I and the first ``sink``."""
+    i = torch.arange(nqb)[:, None]
+    j = torch.arange(nkb)[None, :]
+    m = ((j <= i) & (j > i - window)) | (j < sink)
+    return m.to(torch.uint8).expand(B, Hq, nqb, nkb).contiguous()
+
+
+def block_mask_random(B: int, Hq: int, nqb: int, nkb: int, density: float, seed: int) -> torch.Tensor:
+    """uint8 [B, Hq, nqb, nkb], each block visible with probability ``density`` (seeded)."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    return (torch.rand(B, Hq, nqb, nkb, generator=g) < density).to(torch.uint8)
 
 
 def seqlens_for(B: int, Nk_max: int, seed: int, lo: int = 1024) -> torch.Tensor:
