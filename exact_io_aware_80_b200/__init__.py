@@ -17,14 +17,14 @@ from . import _lib
 from ._lib import (FAError, fa_bwd, fa_bwd_dkdv, fa_bwd_dq, fa_bwd_preprocess, fa_bwd_workspace_bytes,  # noqa: F401
                    fa_decode_chunk, fa_decode_combine, fa_decode_num_splits, fa_decode_splitkv,
                    fa_decode_workspace_bytes, fa_fp8_quantize_qk, fa_fp8_quantize_v, fa_fp8_v_workspace_bytes, fa_fwd,
-                   fa_fwd_fp8, fa_get_device_status, fa_version)
+                   fa_fwd_blocksparse, fa_fwd_fp8, fa_get_device_status, fa_version)
 
 __all__ = [
     "attention_fwd", "attention_bwd", "decode", "decode_splitkv", "decode_combine", "device_status",
     "fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq", "fa_decode_splitkv", "fa_decode_combine", "fa_decode_num_splits",
     "fa_decode_workspace_bytes", "fa_bwd_workspace_bytes", "fa_decode_chunk", "fa_get_device_status",
     "fp8_quantize_qk", "fp8_quantize_v", "attention_fwd_fp8", "fa_fp8_quantize_qk", "fa_fp8_quantize_v",
-    "fa_fp8_v_workspace_bytes", "fa_fwd_fp8", "FAError",
+    "fa_fp8_v_workspace_bytes", "fa_fwd_fp8", "attention_fwd_blocksparse", "fa_fwd_blocksparse", "FAError",
 ]
 
 
@@ -67,6 +67,25 @@ def attention_fwd(q, k, v, causal: bool = False, scale: float | None = None, out
     fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
            causal, scale, _dt(q), _stream(dev))
     return o, l
+
+
+def attention_fwd_blocksparse(q, k, v, block_mask, causal: bool = False, scale: float | None = None):
+    """O, LSE of attention restricted to a 128 x 128 block pattern, via ``fa_fwd_blocksparse``.
+
+    ``block_mask``: uint8 CUDA tensor [B, Hq, ceil(Nq/128), ceil(Nk/128)], nonzero = computed.
+    """
+    torch = _torch()
+    dev = _dev(q, k, v, block_mask)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    if block_mask.dtype != torch.uint8 or tuple(block_mask.shape) != (B, Hq, -(-Nq // 128), -(-Nk // 128)):
+        raise ValueError("block_mask must be uint8 [B, Hq, ceil(Nq/128), ceil(Nk/128)]")
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, Nq, device=dev, dtype=torch.float32)
+    fa_fwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), block_mask.data_ptr(),
+                       B, Hq, Hkv, Nq, Nk, d, causal, scale, _dt(q), _stream(dev))
+    return o, lse
 
 
 def fp8_quantize_qk(x, signs=None):

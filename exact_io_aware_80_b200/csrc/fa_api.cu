@@ -123,6 +123,20 @@ fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const
   return from_cuda(fa::launch_fwd_fp8_sm100(a, static_cast<cudaStream_t>(stream)));
 }
 
+fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                             const uint8_t* block_mask, int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                             float scale, fa_dtype dt, fa_stream_t stream) {
+  if (!q || !k || !v || !o || !lse || !block_mask) return FA_ERR_INVALID;
+  fa_status st = check_shape(B, Hq, Hkv, Nq, Nk, d, causal, dt);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse)) return FA_ERR_ALIGN;
+  fa::AttnArgs a{q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal ? 1 : 0, scale, dt == FA_BF16 ? 1 : 0, status_ptr(),
+                 block_mask};
+  if (!a.status) return FA_ERR_CUDA;
+  if (!fa::fwd_sm100_supported(a)) return FA_ERR_CUDA;
+  return from_cuda(fa::launch_fwd_sm100(a, static_cast<cudaStream_t>(stream)));
+}
+
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq) {
   if (B < 1 || Hq < 1 || Nq < 1) return 0;
   return (size_t)B * Hq * Nq * sizeof(float);

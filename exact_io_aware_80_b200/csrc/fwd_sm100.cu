@@ -37,6 +37,13 @@
 // per instruction), every block's scores are scaled by the Q and K block
 // scales, P is rounded to E4M3 for the P V product, and the epilogue applies
 // V's scale.
+//
+// Instantiated with SPARSE, it is block-sparse attention ("FlashAttention-2
+// (KO)", FA-1 results: the IO-aware kernel extended with a block-sparse
+// pattern): a uint8 table [B, Hq, ceil(Nq/128), ceil(Nk/128)] marks the
+// 128 x 128 blocks that are computed.  A work tile visits only the K/V tiles
+// that either of its query tiles marks, a query tile masks the blocks it does
+// not mark, and a work tile with none writes O = 0 and LSE = -inf directly.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -104,7 +111,8 @@ struct Params {
   const float* q_scale;
   const float* k_scale;
   const float* v_scale;
-  int nqb, nkb;
+  int nqb, nkb;  // 128-row blocks of Nq and Nk (FP8 scales and the block-sparse table)
+  const uint8_t* block_mask;  // block-sparse only: [B, Hq, nqb, nkb], nonzero = computed
 };
 
 // Work tile w of the persistent schedule: row block, query head, batch.  Causal
@@ -130,7 +138,7 @@ __device__ __forceinline__ Work work_at(const Params& p, int w) {
   return x;
 }
 
-template <typename T, int D, bool CAUSAL, bool F8>
+template <typename T, int D, bool CAUSAL, bool F8, bool SPARSE>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, Params p) {
@@ -148,6 +156,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int m0 = mblk * (kTiles * kBM);
     const int n_end = CAUSAL ? min(p.Nk, m0 + kTiles * kBM + off) : p.Nk;
     return (n_end + kBN - 1) / kBN;
+  };
+  // block-sparse: the table row of query tile t of a work tile (null past Nq), and the first
+  // K/V tile >= j below nblk that either query tile marks (j itself for dense attention)
+  auto mask_row = [&](const Work& x, int t) -> const uint8_t* {
+    const int qb = kTiles * x.mblk + t;
+    return qb < p.nqb ? p.block_mask + (((long)x.b * p.Hq + x.hq) * p.nqb + qb) * p.nkb : nullptr;
+  };
+  auto next_vis = [&](const Work& x, int j, int nblk) {
+    if constexpr (SPARSE) {
+      const uint8_t* r0 = mask_row(x, 0);
+      const uint8_t* r1 = mask_row(x, 1);
+      while (j < nblk && !(r0[j] || (r1 && r1[j]))) ++j;
+    }
+    return j;
   };
 
   if (tid == 0) {
@@ -183,13 +205,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       int last_u[kStages] = {-1, -1};
       int last_q = -1;
       int g = 0;  // K/V tiles loaded so far by this CTA (ring position)
+      int we = 0;  // work tiles with at least one K/V tile so far (the per-work-tile barrier phases)
       for (int wl = 0, w = work_index(0); w < p.num_work; w = work_index(++wl)) {
         const Work x = work_at<CAUSAL>(p, w);
         const int hk = x.hq / (p.Hq / p.Hkv);
         const int m0 = x.mblk * (kTiles * kBM);
         const int nblk = blocks_of(x.mblk);
+        if constexpr (SPARSE) {
+          if (next_vis(x, 0, nblk) >= nblk) continue;  // nothing to load: the softmax warps write zeros
+        } else {
+          we = wl;  // every dense work tile visits a K/V tile
+        }
         // the previous tile's last score MMAs must have read Q before it is replaced
-        if (wl > 0 && !mbar_wait(bar(L::kBarQEmpty), (wl - 1) & 1, abort_flag, p.status)) break;
+        if (we > 0 && !mbar_wait(bar(L::kBarQEmpty), (we - 1) & 1, abort_flag, p.status)) break;
         mbar_expect_tx(bar(L::kBarQ), kTiles * L::kTile);
 #pragma unroll
         for (int t = 0; t < kTiles; ++t) {
@@ -202,9 +230,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                           m0 + t * kBM, x.b);
           }
         }
-        last_q = wl;
+        last_q = we++;
         bool stop = false;
-        for (int j = 0; j < nblk; ++j, ++g) {
+        for (int j = next_vis(x, 0, nblk); j < nblk; j = next_vis(x, j + 1, nblk), ++g) {
           const int st = g & 1, u = g >> 1;
           if (u > 0 && !mbar_wait(bar(L::kBarKEmpty + st), (u - 1) & 1, abort_flag, p.status)) {
             stop = true;
@@ -292,9 +320,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       bool ok = true;
       int g = 0;  // K/V tiles consumed so far by this CTA; S/P barriers complete once per tile
+      int we = 0;  // work tiles with at least one K/V tile so far
       for (int wl = 0, w = work_index(0); ok && w < p.num_work; w = work_index(++wl)) {
-        const int nblk = blocks_of(work_at<CAUSAL>(p, w).mblk);
-        ok = mbar_wait(bar(L::kBarQ), wl & 1, abort_flag, p.status) &&
+        const Work x = work_at<CAUSAL>(p, w);
+        const int nblk = blocks_of(x.mblk);
+        const int j0 = next_vis(x, 0, nblk);
+        if constexpr (SPARSE) {
+          if (j0 >= nblk) continue;
+        } else {
+          we = wl;
+        }
+        ok = mbar_wait(bar(L::kBarQ), we & 1, abort_flag, p.status) &&
              mbar_wait(bar(L::kBarKFull + (g & 1)), (g >> 1) & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
@@ -304,18 +340,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         qk(1, g & 1);
         mma_commit(bar(L::kBarS + 1));
         mma_commit(bar(L::kBarKEmpty + (g & 1)));
-        if (nblk == 1) mma_commit(bar(L::kBarQEmpty));
-        for (int j = 0; j < nblk; ++j, ++g) {
+        if (next_vis(x, j0 + 1, nblk) >= nblk) mma_commit(bar(L::kBarQEmpty));
+        for (int j = j0; j < nblk; ++g) {
+          const int jn = next_vis(x, j + 1, nblk);  // the next K/V tile of this work tile
           const int st = g & 1, u = g >> 1;
-          const bool more = j + 1 < nblk;
+          const bool more = jn < nblk;
           const int st1 = (g + 1) & 1, u1 = (g + 1) >> 1;
           ok = mbar_wait(bar(L::kBarVFull + st), u & 1, abort_flag, p.status) &&
                mbar_wait(bar(L::kBarP + 0), g & 1, abort_flag, p.status);
           // the first PV of a tile overwrites O_0: the previous tile's epilogue must have read it
-          if (ok && j == 0 && wl > 0) ok = mbar_wait(bar(L::kBarOFree + 0), (wl - 1) & 1, abort_flag, p.status);
+          if (ok && j == j0 && we > 0) ok = mbar_wait(bar(L::kBarOFree + 0), (we - 1) & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
-          pv(0, st, j == 0);
+          pv(0, st, j == j0);
           if (!more) mma_commit(bar(L::kBarO + 0));
           if (more) {
             ok = mbar_wait(bar(L::kBarKFull + st1), u1 & 1, abort_flag, p.status);
@@ -325,19 +362,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(bar(L::kBarS + 0));
           }
           ok = mbar_wait(bar(L::kBarP + 1), g & 1, abort_flag, p.status);
-          if (ok && j == 0 && wl > 0) ok = mbar_wait(bar(L::kBarOFree + 1), (wl - 1) & 1, abort_flag, p.status);
+          if (ok && j == j0 && we > 0) ok = mbar_wait(bar(L::kBarOFree + 1), (we - 1) & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
-          pv(1, st, j == 0);
+          pv(1, st, j == j0);
           if (!more) mma_commit(bar(L::kBarO + 1));
           mma_commit(bar(L::kBarVEmpty + st));
           if (more) {
             qk(1, st1);
             mma_commit(bar(L::kBarS + 1));
             mma_commit(bar(L::kBarKEmpty + st1));
-            if (j + 2 == nblk) mma_commit(bar(L::kBarQEmpty));  // last score MMAs of this tile issued
+            if (next_vis(x, jn + 1, nblk) >= nblk) mma_commit(bar(L::kBarQEmpty));  // last score MMAs issued
           }
+          j = jn;
         }
+        ++we;
       }
       // no MMA may still run when TMEM is released
       mma_commit(bar(L::kBarDrain));
@@ -355,6 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.scale_log2;
     bool ok = true;
     int g = 0;  // K/V tiles processed so far by this CTA
+    int we = 0;  // work tiles with at least one K/V tile so far
     for (int wl = 0, w = work_index(0); ok && w < p.num_work; w = work_index(++wl)) {
       const Work x = work_at<CAUSAL>(p, w);
       const int h = x.hq, b = x.b;
@@ -362,11 +402,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nblk = blocks_of(x.mblk);
       const int row_first = m0 + t * kBM;
       const int row = row_first + wq * 32 + lane;
+      const int j0 = next_vis(x, 0, nblk);
+      if constexpr (SPARSE) {
+        if (j0 >= nblk) {
+          // block-sparse work tile with no K/V tile: every row attends to nothing
+          if (row < p.Nq) {
+            uint4* orow =
+                reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + (((long)b * p.Nq + row) * p.Hq + h) * D);
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) orow[i] = make_uint4(0u, 0u, 0u, 0u);
+            p.lse[((long)b * p.Hq + h) * p.Nq + row] = -INFINITY;
+          }
+          continue;
+        }
+      } else {
+        we = wl;
+      }
+      const uint8_t* mrow = nullptr;  // this query tile's block-sparse table row
+      if constexpr (SPARSE) mrow = mask_row(x, t);
       const int hk = h / (p.Hq / p.Hkv);
       float cq = c;  // FP8: times the Q tile's block scale
       if constexpr (F8) cq = c * p.q_scale[((long)b * p.Hq + h) * p.nqb + min(row_first / kBM, p.nqb - 1)];
       float m_ref = -INFINITY, l = 0.f;
-        for (int j = 0; j < nblk; ++j, ++g) {
+      for (int j = j0; j < nblk; j = next_vis(x, j + 1, nblk), ++g) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + t), g & 1, abort_flag, p.status));
         if (!ok) break;
         tc_fence_after();
@@ -393,8 +451,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float cj = cq;  // FP8: times the K block's scale
         if constexpr (F8) cj = cq * p.k_scale[((long)b * p.Hkv + hk) * p.nkb + j];
         const int kbase = j * kBN;
-        if (kbase + kBN > p.Nk || (CAUSAL && kbase + kBN - 1 > row_first + off)) {
-          int lim = p.Nk - kbase;
+        bool on = true;  // block-sparse: this query tile computes block (., j)
+        if constexpr (SPARSE) on = mrow && mrow[j];
+        if (!on || kbase + kBN > p.Nk || (CAUSAL && kbase + kBN - 1 > row_first + off)) {
+          int lim = on ? p.Nk - kbase : 0;
           if (CAUSAL) lim = min(lim, row + off + 1 - kbase);
 #pragma unroll
           for (int i = 0; i < kBN; ++i)
@@ -440,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         l += (rs0.x + rs0.y) + (rs1.x + rs1.y);
-        if (__any_sync(0xffffffffu, resc && j > 0)) {
+        if (__any_sync(0xffffffffu, resc && j > j0)) {
 #pragma unroll
           for (int q = 0; q < D / 32; ++q) {
             uint32_t r[32];
@@ -456,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(L::kBarP + t));
       }
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarO + t), wl & 1, abort_flag, p.status));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarO + t), we & 1, abort_flag, p.status));
       uint32_t r[D];
       if (ok) {
         // O_t: TMEM -> registers, then hand the TMEM columns back to the MMA thread at once
@@ -470,16 +530,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(L::kBarOFree + t));
         // the stage buffer alternates tile 0, tile 1, tile 0 (next work tile), ...
         if (t == 1)
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarStageDone + 0), wl & 1, abort_flag, p.status));
-        else if (wl > 0)
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarStageDone + 1), (wl - 1) & 1, abort_flag, p.status));
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarStageDone + 0), we & 1, abort_flag, p.status));
+        else if (we > 0)
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarStageDone + 1), (we - 1) & 1, abort_flag, p.status));
       }
       if (ok) {
         // O / l as 16-bit into the stage buffer, laid out as the TMA box expects: 64-column
         // panels of 128-byte rows, 16-byte chunk c of row r at chunk c ^ (r & 7)
         float num = 1.f;  // FP8: V's scale
         if constexpr (F8) num = p.v_scale[(long)b * p.Hkv + hk];
-        const float inv = l > 0.f ? num / l : 0.f;
+        // block-sparse: a row that saw no visible key keeps m_ref = -inf (its l holds only the
+        // clamped polynomial exp2 of -inf): O = 0 and LSE = -inf
+        const bool any = SPARSE ? (l > 0.f && m_ref != -INFINITY) : l > 0.f;
+        const float inv = any ? num / l : 0.f;
         const int rr = wq * 32 + lane;
         const uint32_t srow = sb + L::kOffStage + rr * 128;
         auto o2 = [&](int i) { return Elem<T>::pack(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv); };
@@ -489,10 +552,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                        o2(8 * c + 4), o2(8 * c + 6));
         fence_proxy_async_smem();
         mbar_arrive(bar(L::kBarStageFull + t));
-        if (row < p.Nq) p.lse[((long)b * p.Hq + h) * p.Nq + row] = l > 0.f ? (m_ref + lg2(l)) * kLn2 : -INFINITY;
+        if (row < p.Nq) p.lse[((long)b * p.Hq + h) * p.Nq + row] = any ? (m_ref + lg2(l)) * kLn2 : -INFINITY;
         if (wq == 0 && lane == 0) {
           // one thread of the tile stores it; rows past Nq are clipped by the tensor map
-          ok = mbar_wait(bar(L::kBarStageFull + t), wl & 1, abort_flag, p.status);
+          ok = mbar_wait(bar(L::kBarStageFull + t), we & 1, abort_flag, p.status);
           if (ok) {
 #pragma unroll
             for (int pn = 0; pn < D / 64; ++pn)
@@ -504,6 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ok = __all_sync(0xffffffffu, ok);
       }
+      ++we;
     }
     // stores must be complete before the CTA exits
     if (wq == 0 && lane == 0) bulk_wait_all();
@@ -532,8 +596,17 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   const long long num_work = (long long)num_mblk * a.Hq * a.B;
   if (num_work > (1ll << 31) - 1) return cudaErrorInvalidValue;
   Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, a.scale * kLog2e, a.status, num_mblk, (int)num_work,
-           nullptr, nullptr, nullptr, 0, 0};
-  auto kern = fwd_sm100_kernel<T, D, CAUSAL, false>;
+           nullptr, nullptr, nullptr, (a.Nq + kBM - 1) / kBM, (a.Nk + kBN - 1) / kBN, a.block_mask};
+  if (a.block_mask) {
+    auto kern = fwd_sm100_kernel<T, D, CAUSAL, false, true>;
+    const int smem = Smem<D, false>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)std::min<long long>(num_work, device_sm_count());
+    kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mo, p);
+    return cudaGetLastError();
+  }
+  auto kern = fwd_sm100_kernel<T, D, CAUSAL, false, false>;
   const int smem = Smem<D, false>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -565,8 +638,8 @@ cudaError_t launch_f8(const Fp8AttnArgs& a, cudaStream_t s) {
   if (num_work > (1ll << 31) - 1) return cudaErrorInvalidValue;
   const float sl2 = a.scale * kLog2e / (a.rotated ? (float)D : 1.f);
   Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, sl2, a.status, num_mblk, (int)num_work,
-           a.q_scale, a.k_scale, a.v_scale, (a.Nq + kBM - 1) / kBM, (a.Nk + kBN - 1) / kBN};
-  auto kern = fwd_sm100_kernel<T, D, CAUSAL, true>;
+           a.q_scale, a.k_scale, a.v_scale, (a.Nq + kBM - 1) / kBM, (a.Nk + kBN - 1) / kBN, nullptr};
+  auto kern = fwd_sm100_kernel<T, D, CAUSAL, true, false>;
   const int smem = Smem<D, true>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

@@ -19,6 +19,7 @@ struct AttnArgs {
   float scale;
   int bf16;  // 1: bf16, 0: fp16
   int* status;
+  const uint8_t* block_mask = nullptr;  // block-sparse forward: [B, Hq, ceil(Nq/128), ceil(Nk/128)]
 };
 
 struct BwdArgs {

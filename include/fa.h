@@ -41,6 +41,7 @@
 #define FA_H_
 
 #include <stddef.h>
+#include <stdint.h>
 
 #ifdef __cplusplus
 extern "C" {
@@ -183,6 +184,19 @@ int fa_decode_chunk(int Nk_max, int num_splits);
 fa_status fa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const int* seqlens_k,
                             void* o, float* lse, int B, int Hq, int Hkv, int Nk_max, int d, float scale,
                             int num_splits, fa_dtype dt, fa_stream_t stream);
+
+/*
+ * Block-sparse forward ("FlashAttention-2 (KO)", FA-1 results: the IO-aware
+ * kernel extended with a block-sparse pattern).  block_mask: device uint8
+ * [B, Hq, ceil(Nq / 128), ceil(Nk / 128)]; entry (b, h, I, J) nonzero means
+ * queries 128 I .. 128 I + 127 may attend to keys 128 J .. 128 J + 127
+ * (intersected with the causal rule when causal).  Blocks not marked are
+ * skipped; a row with no visible key gets O = 0 and LSE = -inf.  Otherwise as
+ * fa_fwd (layouts, GQA, alignment, errors).
+ */
+fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                             const uint8_t* block_mask, int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                             float scale, fa_dtype dt, fa_stream_t stream);
 
 /* ------------------------------------------------------------------------------
  * FP8 forward pass ("FlashAttention-2 (KO)", FA-3 paragraph: low-precision FP8

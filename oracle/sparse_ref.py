@@ -24,7 +24,8 @@ import numpy as np
 
 from .attn_ref import _check_shapes, _f64, scores, softmax_rows, visible_mask
 
-__all__ = ["BLOCK", "expand_block_mask", "attention_fwd_blocksparse", "blocksparse_flops"]
+__all__ = ["BLOCK", "expand_block_mask", "attention_fwd_blocksparse", "attention_fwd_blocksparse_rows",
+           "blocksparse_flops"]
 
 BLOCK = 128
 
@@ -54,6 +55,18 @@ def attention_fwd_blocksparse(q, k, v, block_mask, causal: bool, scale: float, h
         O[b, :, h, :] = P @ v[b, :, h // G, :]
         LSE[b, h, :] = lse
     return O, LSE
+
+
+def attention_fwd_blocksparse_rows(q, k, v, block_mask, causal: bool, scale: float, b: int, h: int, rows):
+    """O [len(rows), d] and LSE [len(rows)] of selected query rows of one (b, h_q)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Nq, Nk, Hq, Hkv, d = _check_shapes(q, k, v)
+    rows = np.asarray(rows, dtype=np.int64)
+    mask = expand_block_mask(np.asarray(block_mask)[b, h], Nq, Nk, causal)[rows]
+    hk = h // (Hq // Hkv)
+    S = scores(q[b, rows, h, :], k[b, :, hk, :], scale, mask)
+    P, lse = softmax_rows(S)
+    return P @ v[b, :, hk, :], lse
 
 
 def blocksparse_flops(block_mask, Nq: int, Nk: int, d: int, causal: bool) -> float:

@@ -153,3 +153,17 @@ def test_fp8_entry_points_reject_bad_arguments(lib):
     bad = list(base)
     bad[4] = FAKE + 4  # v8t misaligned
     assert lib.fa_fwd_fp8(*bad) == -3
+
+
+def test_blocksparse_rejects_bad_arguments(lib):
+    # q, k, v, o, lse, mask, B, Hq, Hkv, Nq, Nk, d, causal, scale, dt, stream
+    base = [FAKE] * 6 + [1, 4, 2, 8, 8, 128, 0, 0.1, 1, None]
+    bad = list(base)
+    bad[5] = 0  # no mask
+    assert lib.fa_fwd_blocksparse(*bad) == -1
+    bad = list(base)
+    bad[11] = 80
+    assert lib.fa_fwd_blocksparse(*bad) == -2
+    bad = list(base)
+    bad[0] = FAKE + 2
+    assert lib.fa_fwd_blocksparse(*bad) == -3

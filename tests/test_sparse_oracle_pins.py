@@ -76,3 +76,13 @@ def test_flops_count_visible_pairs():
     bm = np.array([[[[1, 0], [1, 1]]]], np.uint8)
     assert sp.blocksparse_flops(bm, 256, 256, 8, False) == 4 * 8 * (3 * 128 * 128)
     assert sp.blocksparse_flops(bm, 256, 256, 8, True) == 4 * 8 * (128 * 129 // 2 + 128 * 128 + 128 * 129 // 2)
+
+
+def test_rows_variant_equals_full():
+    q, k, v = rnd((2, 300, 4, 16), 20), rnd((2, 400, 2, 16), 21), rnd((2, 400, 2, 16), 22)
+    bm = (np.random.default_rng(23).random((2, 4, 3, 4)) < 0.5).astype(np.uint8)
+    O, L = sp.attention_fwd_blocksparse(q, k, v, bm, True, 0.25)
+    rows = [0, 5, 127, 128, 299]
+    Or, Lr = sp.attention_fwd_blocksparse_rows(q, k, v, bm, True, 0.25, 1, 3, rows)
+    np.testing.assert_array_equal(Or, O[1, rows, 3, :])
+    np.testing.assert_array_equal(Lr, L[1, 3, rows])
