@@ -272,6 +272,8 @@ def run_ours(args):
                                                     peaks_kind)
     fp8 = None if args.no_fp8 else run_fp8(args, torch, fa, _lib, workloads, w, q, k, v, dev, stream, world, peaks,
                                            peaks_kind)
+    sparse = None if args.no_sparse else run_blocksparse(args, torch, fa, _lib, workloads, w, q, k, v, dev, stream,
+                                                         world, peaks, peaks_kind)
     e2e = run_e2e(args, torch, fa, w, q, k, v, do, dev, stream, world, F) if not args.no_e2e else None
 
     cpu = None
@@ -296,6 +298,7 @@ def run_ours(args):
                   "per_kernel_ms": {kk: round(vv, 4) for kk, vv in per.items()}},
         "decode": decode,
         "fp8": fp8,
+        "blocksparse": sparse,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -435,6 +438,56 @@ def run_fp8(args, torch, fa, _lib, workloads, w, q, k, v, dev, stream, world, pe
             "gpu_launches": 5 * K}
 
 
+def run_blocksparse(args, torch, fa, _lib, workloads, w, q, k, v, dev, stream, world, peaks, peaks_kind):
+    """Block-sparse forward on the same GQA inputs: causal, local window of 8 key blocks + the first block."""
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.Nq, w.d
+    nb = (N + 127) // 128
+    window = 8
+    bm = workloads.block_mask_local(B, Hq, nb, nb, window=window, sink=1).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, N, device=dev, dtype=torch.float32)
+    sh = stream.cuda_stream
+
+    def step():
+        _lib.fa_fwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), bm.data_ptr(),
+                                B, Hq, Hkv, N, N, d, 1, w.scale, _lib.FA_BF16, sh)
+
+    for _ in range(args.warmup):
+        step()
+    K = args.steps
+    barrier(torch, world)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(K):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(torch, world)
+    ms = max_over_ranks(torch, world, t0.elapsed_time(t1)) / K
+    if fa.device_status() != 0:
+        raise RuntimeError("kernel status word set during the block-sparse section")
+    # FLOPs of the visible pairs (4 d per pair): per query block I, causal diagonal block plus full blocks
+    pairs = 0
+    for I in range(nb):
+        js = set(range(max(0, I - window + 1), I + 1)) | {0}
+        for J in js:
+            pairs += 128 * 129 // 2 if J == I else 128 * 128
+    F = 4.0 * d * pairs * B * Hq
+    key = "bf16_tflops_sustained" if ms * K >= 2000 else "bf16_tflops"
+    peak = float(peaks.get(key, FALLBACK_PEAKS[key]))
+    ach = F / (ms * 1e-3) / 1e12
+    dense = attn_flops(B, Hq, N, N, d, True)
+    return {"workload": f"block-sparse forward, causal, local window {window} blocks + first block (128 x 128 blocks): "
+                        f"B={B} Hq={Hq} Hkv={Hkv} N={N} d={d} bf16",
+            "density_vs_causal": round(F / dense, 4), "ms_per_step": round(ms, 4),
+            "value": round(world * ach, 1), "unit": "TFLOP/s (visible pairs)",
+            "roofline": {"bound": "tensor", "kernel": "fwd_sm100_kernel (SPARSE)", "achieved": round(ach, 1),
+                         "peak": peak, "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                         "peak_source": f"{peaks_kind} {key}", "algorithmic_flops_per_launch": F},
+            "gpu_launches": K}
+
+
 def run_e2e(args, torch, fa, w, q, k, v, do, dev, stream, world, F):
     """Same step through the public Python API with host buffers: pinned H2D of
     q, k, v, dO, forward, backward, D2H of dQ, dK, dV, all inside the timed region."""
@@ -563,6 +616,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode section (profiling runs)")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 forward section (profiling runs)")
+    ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse section (profiling runs)")
     ap.add_argument("--decode-b", type=int, default=0,
                     help="override B of the decode workload (profiling runs on a smaller case)")
     ap.add_argument("--seq", type=int, default=0,
