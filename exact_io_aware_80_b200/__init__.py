@@ -17,14 +17,15 @@ from . import _lib
 from ._lib import (FAError, fa_bwd, fa_bwd_dkdv, fa_bwd_dq, fa_bwd_preprocess, fa_bwd_workspace_bytes,  # noqa: F401
                    fa_decode_chunk, fa_decode_combine, fa_decode_num_splits, fa_decode_splitkv,
                    fa_decode_workspace_bytes, fa_fp8_quantize_qk, fa_fp8_quantize_v, fa_fp8_v_workspace_bytes, fa_fwd,
-                   fa_fwd_blocksparse, fa_fwd_fp8, fa_get_device_status, fa_version)
+                   fa_bwd_dropout, fa_fwd_blocksparse, fa_fwd_dropout, fa_fwd_fp8, fa_get_device_status, fa_version)
 
 __all__ = [
     "attention_fwd", "attention_bwd", "decode", "decode_splitkv", "decode_combine", "device_status",
     "fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq", "fa_decode_splitkv", "fa_decode_combine", "fa_decode_num_splits",
     "fa_decode_workspace_bytes", "fa_bwd_workspace_bytes", "fa_decode_chunk", "fa_get_device_status",
     "fp8_quantize_qk", "fp8_quantize_v", "attention_fwd_fp8", "fa_fp8_quantize_qk", "fa_fp8_quantize_v",
-    "fa_fp8_v_workspace_bytes", "fa_fwd_fp8", "attention_fwd_blocksparse", "fa_fwd_blocksparse", "FAError",
+    "fa_fp8_v_workspace_bytes", "fa_fwd_fp8", "attention_fwd_blocksparse", "fa_fwd_blocksparse",
+    "attention_fwd_dropout", "attention_bwd_dropout", "fa_fwd_dropout", "fa_bwd_dropout", "FAError",
 ]
 
 
@@ -67,6 +68,37 @@ def attention_fwd(q, k, v, causal: bool = False, scale: float | None = None, out
     fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
            causal, scale, _dt(q), _stream(dev))
     return o, l
+
+
+def attention_fwd_dropout(q, k, v, p_drop: float, seed: int, offset: int = 0, causal: bool = False,
+                          scale: float | None = None):
+    """O, LSE with dropout on P (mask from Philox4x32-10, see include/fa.h), via ``fa_fwd_dropout``."""
+    torch = _torch()
+    dev = _dev(q, k, v)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, Nq, device=dev, dtype=torch.float32)
+    fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
+                   causal, scale, p_drop, seed, offset, _dt(q), _stream(dev))
+    return o, lse
+
+
+def attention_bwd_dropout(q, k, v, o, do, lse, p_drop: float, seed: int, offset: int = 0, causal: bool = False,
+                          scale: float | None = None):
+    """dQ, dK, dV for attention_fwd_dropout with the same p_drop, seed and offset, via ``fa_bwd_dropout``."""
+    torch = _torch()
+    dev = _dev(q, k, v, o, do, lse)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa_bwd_workspace_bytes(B, Hq, Nq), device=dev, dtype=torch.uint8)
+    fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+                   dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, Nk, d, causal, scale, p_drop, seed,
+                   offset, _dt(q), _stream(dev))
+    return dq, dk, dv
 
 
 def attention_fwd_blocksparse(q, k, v, block_mask, causal: bool = False, scale: float | None = None):

@@ -40,6 +40,10 @@ SIGNATURES = {
     "fa_decode_chunk": (_I, [_I, _I]),
     "fa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "fa_fwd_blocksparse": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_fwd_dropout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, ctypes.c_uint64, ctypes.c_uint32,
+                            _I, _P]),
+    "fa_bwd_dropout": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F,
+                            ctypes.c_uint64, ctypes.c_uint32, _I, _P]),
     "fa_fp8_quantize_qk": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "fa_fp8_v_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I]),
     "fa_fp8_quantize_v": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
@@ -134,6 +138,18 @@ def fa_decode_splitkv(q, k_cache, v_cache, seqlens_k, B, Hq, Hkv, Nk_max, d, sca
 def fa_decode_combine(workspace, o, lse, seqlens_k, B, Hq, num_splits, d, dt, stream):
     return _check("fa_decode_combine", load().fa_decode_combine(workspace, o, lse, seqlens_k, B, Hq, num_splits, d,
                                                                 dt, stream))
+
+
+def fa_fwd_dropout(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, p_drop, seed, offset, dt, stream):
+    return _check("fa_fwd_dropout", load().fa_fwd_dropout(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, int(causal), scale,
+                                                          p_drop, seed, offset, dt, stream))
+
+
+def fa_bwd_dropout(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, causal, scale, p_drop, seed,
+                   offset, dt, stream):
+    return _check("fa_bwd_dropout", load().fa_bwd_dropout(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, Hq, Hkv, Nq,
+                                                          Nk, d, int(causal), scale, p_drop, seed, offset, dt,
+                                                          stream))
 
 
 def fa_fwd_blocksparse(q, k, v, o, lse, block_mask, B, Hq, Hkv, Nq, Nk, d, causal, scale, dt, stream):

@@ -25,6 +25,10 @@
 //   dP = dO V^T, then dQ += dS K; S for tile j+2 is queued behind dQ_j so the
 //   exponentials of one tile overlap the MMAs of the next.
 //
+// With DROP both kernels regenerate the forward pass's dropout mask (Philox
+// words from the same counters, common.cuh): dV uses P * M, and dS =
+// P * (M * dP / (1 - p) - D); dV is scaled by 1 / (1 - p) when stored.
+//
 // Every mbarrier wait is bounded (sm100.cuh) and the roles drain in-flight
 // copies and MMAs before tensor memory is released.
 #include <cuda.h>
@@ -54,6 +58,7 @@ struct Params {
   float scale;
   float scale_log2;
   int* status;
+  Dropout drop;  // DROP only
 };
 
 // Store one 128-byte-aligned row segment of D 16-bit values from fp32 TMEM columns.
@@ -105,9 +110,10 @@ __device__ __forceinline__ void load_row128(uint32_t taddr, float (&s)[kT]) {
 // first 64 columns starting at `tds`; reads dP 32 columns at a time from `tdp`.
 // The caller passes d negated: per column (dcol[c] = -D_c) or per row (drow = -D_i).
 // When tds == tdp the writes trail the reads (columns 16c.. after 32c.. are read).
-template <typename T, bool PER_COL_D>
+// With DROP, element c uses M * dP / (1 - p): keep bit c of `keep` (128 bits) and inv_keep.
+template <typename T, bool PER_COL_D, bool DROP = false>
 __device__ __forceinline__ void write_ds(uint32_t tdp, uint32_t tds, const float (&p)[kT], const float* dcol,
-                                         float drow) {
+                                         float drow, const uint32_t (&keep)[4] = {}, float inv_keep = 1.f) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint32_t r[32];
@@ -119,8 +125,12 @@ __device__ __forceinline__ void write_ds(uint32_t tdp, uint32_t tds, const float
     for (int i = 0; i < 16; ++i) {
       const int c0 = q * 32 + 2 * i;
       const float2 nd = PER_COL_D ? reinterpret_cast<const float2*>(dcol)[c0 >> 1] : make_float2(drow, drow);
-      const float2 ds = __fmul2_rn(make_float2(p[c0], p[c0 + 1]),
-                                   __fadd2_rn(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), nd));
+      float2 dp = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+      if constexpr (DROP) {
+        dp.x = (keep[c0 >> 5] >> (c0 & 31)) & 1u ? dp.x * inv_keep : 0.f;
+        dp.y = (keep[c0 >> 5] >> ((c0 + 1) & 31)) & 1u ? dp.y * inv_keep : 0.f;
+      }
+      const float2 ds = __fmul2_rn(make_float2(p[c0], p[c0 + 1]), __fadd2_rn(dp, nd));
       pk[i] = Elem<T>::pack(ds.x, ds.y);
     }
     tmem_st16(tds + q * 16, pk);
@@ -149,7 +159,7 @@ struct DkdvSmem {
 // TMEM columns: S^T / P^T, dP^T / dS^T, dV, dK
 constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256, kColDK = 384;
 
-template <typename T, int D, bool CAUSAL>
+template <typename T, int D, bool CAUSAL, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -341,12 +351,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int cc = 0; cc < kT; ++cc)
           if (cc < lim) pv[cc] = 0.f;
       }
+      uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit cc = (query i0 + cc, this key) kept
+      if constexpr (DROP) {
+        const uint32_t bh = (uint32_t)(b * p.Hq + hk * G + t / per_head), jp = (uint32_t)key >> 1;
+        const bool kodd = key & 1;
+#pragma unroll
+        for (int wd = 0; wd < 4; ++wd) {
+          uint32_t m = 0;
+#pragma unroll 1
+          for (int k2 = 0; k2 < 32; k2 += 2) {
+            // the call of the 2 x 2 block (queries i0 + cc, + 1) x (keys 2 jp, 2 jp + 1)
+            const int cc = 32 * wd + k2;
+            const uint4 w = philox4x32_10(jp, (uint32_t)(i0 + cc) >> 1, bh, p.drop.offset, p.drop.seed_lo,
+                                          p.drop.seed_hi);
+            const uint32_t k0b = (kodd ? w.y : w.x) >= p.drop.thr, k1b = (kodd ? w.w : w.z) >= p.drop.thr;
+            m |= (k0b << k2) | (k1b << (k2 + 1));
+          }
+          keep[wd] = m;
+        }
+      }
       {
+        auto pd = [&](int c) { return DROP && !((keep[c >> 5] >> (c & 31)) & 1u) ? 0.f : pv[c]; };
         uint32_t pk0[32], pk1[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          pk0[i] = Elem<T>::pack(pv[2 * i], pv[2 * i + 1]);
-          pk1[i] = Elem<T>::pack(pv[64 + 2 * i], pv[64 + 2 * i + 1]);
+          pk0[i] = Elem<T>::pack(pd(2 * i), pd(2 * i + 1));
+          pk1[i] = Elem<T>::pack(pd(64 + 2 * i), pd(64 + 2 * i + 1));
         }
         tmem_st32(tST + 0, pk0);
         tmem_st32(tST + 32, pk1);
@@ -358,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), t & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
-      write_ds<T, true>(tDPT, tDPT, pv, s_d + buf * kT, 0.f);
+      write_ds<T, true, DROP>(tDPT, tDPT, pv, s_d + buf * kT, 0.f, keep, p.drop.inv_keep);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(L::kBarDS));
@@ -373,7 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const bool valid = key < p.Nk;
       const long row = ((long)b * p.Nk + key) * p.Hkv + hk;
-      store_row<T, D>(tbase + lane_off + kColDV, static_cast<uint16_t*>(p.out1) + row * D, 1.f, valid);
+      store_row<T, D>(tbase + lane_off + kColDV, static_cast<uint16_t*>(p.out1) + row * D,
+                      DROP ? p.drop.inv_keep : 1.f, valid);
       store_row<T, D>(tbase + lane_off + kColDK, static_cast<uint16_t*>(p.out0) + row * D, p.scale, valid);
     }
   }
@@ -408,7 +439,7 @@ struct DqSmem {
 __host__ __device__ constexpr uint32_t col_s(int buf) { return 128u * buf; }
 constexpr uint32_t kColDP = 256, kColDQ = 384;
 
-template <typename T, int D, bool CAUSAL>
+template <typename T, int D, bool CAUSAL, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -575,7 +606,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), j & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
-      write_ds<T, false>(tbase + lane_off + kColDP, tS, pv, nullptr, ndrow);
+      uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit cc = (this query, key kb + cc) kept
+      if constexpr (DROP) {
+        const uint32_t bh = (uint32_t)(b * p.Hq + h), rh = (uint32_t)row >> 1;
+        const bool odd = row & 1;
+#pragma unroll
+        for (int wd = 0; wd < 4; ++wd) {
+          uint32_t m = 0;
+#pragma unroll 1
+          for (int k2 = 0; k2 < 32; k2 += 2) {
+            const int cc = 32 * wd + k2;
+            const uint4 w = philox4x32_10((uint32_t)(kb + cc) >> 1, rh, bh, p.drop.offset, p.drop.seed_lo,
+                                          p.drop.seed_hi);
+            const uint32_t k0b = (odd ? w.z : w.x) >= p.drop.thr, k1b = (odd ? w.w : w.y) >= p.drop.thr;
+            m |= (k0b << k2) | (k1b << (k2 + 1));
+          }
+          keep[wd] = m;
+        }
+      }
+      write_ds<T, false, DROP>(tbase + lane_off + kColDP, tS, pv, nullptr, ndrow, keep, p.drop.inv_keep);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(L::kBarDS));
@@ -612,14 +661,15 @@ bool make_maps(Maps& m, const BwdArgs& a) {
 }
 
 Params params(const BwdArgs& a, void* out0, void* out1) {
-  return Params{a.lse, a.dvec, out0, out1, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, a.scale, a.scale * kLog2e, a.status};
+  return Params{a.lse,  a.dvec,      out0,  out1, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, a.scale, a.scale * kLog2e, a.status,
+                Dropout{a.drop_thr, a.drop_inv_keep, a.seed_lo, a.seed_hi, a.drop_offset}};
 }
 
 template <typename T, int D, bool CAUSAL>
 cudaError_t launch_dkdv(const BwdArgs& a, cudaStream_t s) {
   Maps m;
   if (!make_maps(m, a)) return cudaErrorInvalidValue;
-  auto kern = bwd_dkdv_sm100_kernel<T, D, CAUSAL>;
+  auto kern = a.drop_p > 0.f ? bwd_dkdv_sm100_kernel<T, D, CAUSAL, true> : bwd_dkdv_sm100_kernel<T, D, CAUSAL, false>;
   const int smem = DkdvSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -632,7 +682,7 @@ template <typename T, int D, bool CAUSAL>
 cudaError_t launch_dq(const BwdArgs& a, cudaStream_t s) {
   Maps m;
   if (!make_maps(m, a)) return cudaErrorInvalidValue;
-  auto kern = bwd_dq_sm100_kernel<T, D, CAUSAL>;
+  auto kern = a.drop_p > 0.f ? bwd_dq_sm100_kernel<T, D, CAUSAL, true> : bwd_dq_sm100_kernel<T, D, CAUSAL, false>;
   const int smem = DqSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

@@ -22,6 +22,39 @@ constexpr float kLn2 = 0.6931471805599453f;
 // Device status word codes (mirrors fa_status in fa.h).
 constexpr int kStatusTimeout = -5;
 
+// Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, "Parallel random
+// numbers: as easy as 1, 2, 3", SC 2011): per round, with M0 = 0xD2511F53 and
+// M1 = 0xCD9E8D57, (c0, c1, c2, c3) -> (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2),
+// hi(M0 c0) ^ c3 ^ k1, lo(M0 c0)); the key is bumped by the Weyl constants
+// (0x9E3779B9, 0xBB67AE85) before every round but the first.  Used for the
+// dropout mask, which the backward kernels regenerate from the same counters.
+__device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, uint32_t k0,
+                                               uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t lo0 = c0 * 0xD2511F53u, hi0 = __umulhi(c0, 0xD2511F53u);
+    const uint32_t lo1 = c2 * 0xCD9E8D57u, hi1 = __umulhi(c2, 0xCD9E8D57u);
+    c0 = hi1 ^ c1 ^ k0;
+    c1 = lo1;
+    c2 = hi0 ^ c3 ^ k1;
+    c3 = lo0;
+  }
+  return make_uint4(c0, c1, c2, c3);
+}
+
+// Dropout of one (b, h_q): one Philox call per 2 x 2 block of (query i, key j),
+// counter (j >> 1, i >> 1, b * Hq + h, offset), key = the 64-bit seed; word
+// 2 (i & 1) + (j & 1) decides (i, j): kept iff it is >= thr = floor(p 2^32).
+struct Dropout {
+  uint32_t thr;       // floor(p * 2^32)
+  float inv_keep;     // 1 / (1 - p)
+  uint32_t seed_lo, seed_hi, offset;
+};
+
 // ---------------------------------------------------------------------------
 // element types
 // ---------------------------------------------------------------------------

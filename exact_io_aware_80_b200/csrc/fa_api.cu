@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cmath>
 #include <mutex>
 
 #include "fa.h"
@@ -49,6 +50,34 @@ fa_status check_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
 }
 
 fa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+// Dropout parameters: keep iff the Philox word >= floor(p 2^32), weights scaled by 1 / (1 - p).
+struct DropParams {
+  float p = 0.f;
+  uint32_t thr = 0;
+  float inv_keep = 1.f;
+  uint32_t seed_lo = 0, seed_hi = 0, offset = 0;
+};
+bool make_drop(float p, unsigned long long seed, uint32_t offset, DropParams* out) {
+  if (!(p >= 0.f && p < 1.f)) return false;
+  const double t = std::floor((double)p * 4294967296.0);
+  out->p = p;
+  out->thr = (uint32_t)(t > 4294967295.0 ? 4294967295.0 : t);
+  out->inv_keep = (float)(1.0 / (1.0 - (double)p));
+  out->seed_lo = (uint32_t)(seed & 0xFFFFFFFFull);
+  out->seed_hi = (uint32_t)(seed >> 32);
+  out->offset = offset;
+  return true;
+}
+template <typename A>
+void apply_drop(A& a, const DropParams& d) {
+  a.drop_p = d.p;
+  a.drop_thr = d.thr;
+  a.drop_inv_keep = d.inv_keep;
+  a.seed_lo = d.seed_lo;
+  a.seed_hi = d.seed_hi;
+  a.drop_offset = d.offset;
+}
 
 }  // namespace
 
@@ -123,6 +152,22 @@ fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const
   return from_cuda(fa::launch_fwd_fp8_sm100(a, static_cast<cudaStream_t>(stream)));
 }
 
+fa_status fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                         int Nq, int Nk, int d, int causal, float scale, float p_drop, unsigned long long seed,
+                         uint32_t offset, fa_dtype dt, fa_stream_t stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID;
+  DropParams dp;
+  if (!make_drop(p_drop, seed, offset, &dp)) return FA_ERR_INVALID;
+  fa_status st = check_shape(B, Hq, Hkv, Nq, Nk, d, causal, dt);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse)) return FA_ERR_ALIGN;
+  fa::AttnArgs a{q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal ? 1 : 0, scale, dt == FA_BF16 ? 1 : 0, status_ptr()};
+  apply_drop(a, dp);
+  if (!a.status) return FA_ERR_CUDA;
+  if (!fa::fwd_sm100_supported(a)) return FA_ERR_CUDA;
+  return from_cuda(fa::launch_fwd_sm100(a, static_cast<cudaStream_t>(stream)));
+}
+
 fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
                              const uint8_t* block_mask, int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
                              float scale, fa_dtype dt, fa_stream_t stream) {
@@ -147,7 +192,8 @@ enum { kPre = 1, kDkdv = 2, kDq = 4 };
 
 static fa_status bwd_run(int steps, const void* q, const void* k, const void* v, const void* o, const void* dout,
                          const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv,
-                         int Nq, int Nk, int d, int causal, float scale, fa_dtype dt, fa_stream_t stream) {
+                         int Nq, int Nk, int d, int causal, float scale, fa_dtype dt, fa_stream_t stream,
+                         const DropParams& drop = DropParams{}) {
   const bool pre = steps & kPre, dkdv = steps & kDkdv, dqs = steps & kDq;
   if (!workspace || !dout) return FA_ERR_INVALID;
   if (pre && !o) return FA_ERR_INVALID;
@@ -163,6 +209,7 @@ static fa_status bwd_run(int steps, const void* q, const void* k, const void* v,
   if ((dkdv || dqs) && !fa::tma_available()) return FA_ERR_CUDA;  // the driver lacks the tensor-map encoder
   fa::BwdArgs a{q, k, v, o, dout, lse, dq, dk, dv, static_cast<float*>(workspace), B, Hq, Hkv, Nq, Nk, d,
                 causal ? 1 : 0, scale, dt == FA_BF16 ? 1 : 0, status_ptr()};
+  apply_drop(a, drop);
   if (!a.status) return FA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaSuccess;
@@ -178,6 +225,17 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID;
   return bwd_run(kPre | kDkdv | kDq, q, k, v, o, dout, lse, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, causal,
                  scale, dt, stream);
+}
+
+fa_status fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                         const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv,
+                         int Nq, int Nk, int d, int causal, float scale, float p_drop, unsigned long long seed,
+                         uint32_t offset, fa_dtype dt, fa_stream_t stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID;
+  DropParams dp;
+  if (!make_drop(p_drop, seed, offset, &dp)) return FA_ERR_INVALID;
+  return bwd_run(kPre | kDkdv | kDq, q, k, v, o, dout, lse, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, causal,
+                 scale, dt, stream, dp);
 }
 
 fa_status fa_bwd_preprocess(const void* q, const void* k, const void* v, const void* o, const void* dout,

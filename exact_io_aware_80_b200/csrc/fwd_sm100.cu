@@ -44,6 +44,13 @@
 // 128 x 128 blocks that are computed.  A work tile visits only the K/V tiles
 // that either of its query tiles marks, a query tile masks the blocks it does
 // not mark, and a work tile with none writes O = 0 and LSE = -inf directly.
+//
+// Instantiated with DROP, it applies dropout to P ("FlashAttention 심층 분석",
+// section 2: dropout is one of the fused steps): every 4-key step of the
+// exponentials draws two Philox4x32-10 words per row (common.cuh: one call per
+// 2 x 2 block of query/key pairs) and zeroes the dropped entries of P before
+// the P V product; l keeps the sum of the undropped p, so LSE is that of the
+// scores, and the epilogue multiplies O by 1 / (1 - p).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -113,6 +120,7 @@ struct Params {
   const float* v_scale;
   int nqb, nkb;  // 128-row blocks of Nq and Nk (FP8 scales and the block-sparse table)
   const uint8_t* block_mask;  // block-sparse only: [B, Hq, nqb, nkb], nonzero = computed
+  Dropout drop;               // dropout only
 };
 
 // Work tile w of the persistent schedule: row block, query head, batch.  Causal
@@ -138,7 +146,7 @@ __device__ __forceinline__ Work work_at(const Params& p, int w) {
   return x;
 }
 
-template <typename T, int D, bool CAUSAL, bool F8, bool SPARSE>
+template <typename T, int D, bool CAUSAL, bool F8, bool SPARSE, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, Params p) {
@@ -474,6 +482,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (resc) m_ref = mxs;
         l *= corr;
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+        uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit c = (this row, key kbase + c) kept
+        if constexpr (DROP) {
+          const uint32_t rh = (uint32_t)row >> 1, bh = (uint32_t)(b * p.Hq + h);
+          const bool odd = row & 1;
+#pragma unroll
+          for (int wd = 0; wd < 4; ++wd) {
+            uint32_t m = 0;
+#pragma unroll 1
+            for (int k2 = 0; k2 < 32; k2 += 2) {
+              // the call of the 2 x 2 block (this row's query pair) x (keys kbase + 32 wd + k2, + 1)
+              const uint4 w = philox4x32_10((uint32_t)(kbase + 32 * wd + k2) >> 1, rh, bh, p.drop.offset,
+                                            p.drop.seed_lo, p.drop.seed_hi);
+              const uint32_t k0b = (odd ? w.z : w.x) >= p.drop.thr, k1b = (odd ? w.w : w.y) >= p.drop.thr;
+              m |= (k0b << k2) | (k1b << (k2 + 1));
+            }
+            keep[wd] = m;
+          }
+        }
         const float2 c2 = make_float2(cj, cj), nm2 = make_float2(-mu, -mu);
         float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -486,11 +512,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float2 bb = exp2_pair(__ffma2_rn(make_float2(s[c0 + 2], s[c0 + 3]), c2, nm2), 32 * half + i + 1);
             rs0 = __fadd2_rn(rs0, a);
             rs1 = __fadd2_rn(rs1, bb);
+            float2 ad = a, bd = bb;  // the weights of the P V product
+            if constexpr (DROP) {
+              const uint32_t kw = keep[c0 >> 5], sh = c0 & 31;
+              ad.x = (kw >> sh) & 1u ? a.x : 0.f;
+              ad.y = (kw >> (sh + 1)) & 1u ? a.y : 0.f;
+              bd.x = (kw >> (sh + 2)) & 1u ? bb.x : 0.f;
+              bd.y = (kw >> (sh + 3)) & 1u ? bb.y : 0.f;
+            }
             if constexpr (F8) {
-              pk[i >> 1] = pack_e4m3x4(a.x, a.y, bb.x, bb.y);  // keys c0 .. c0 + 3 in one column
+              pk[i >> 1] = pack_e4m3x4(ad.x, ad.y, bd.x, bd.y);  // keys c0 .. c0 + 3 in one column
             } else {
-              pk[i] = Elem<T>::pack(a.x, a.y);
-              pk[i + 1] = Elem<T>::pack(bb.x, bb.y);
+              pk[i] = Elem<T>::pack(ad.x, ad.y);
+              pk[i + 1] = Elem<T>::pack(bd.x, bd.y);
             }
           }
           if constexpr (F8) {
@@ -537,8 +571,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         // O / l as 16-bit into the stage buffer, laid out as the TMA box expects: 64-column
         // panels of 128-byte rows, 16-byte chunk c of row r at chunk c ^ (r & 7)
-        float num = 1.f;  // FP8: V's scale
+        float num = 1.f;  // FP8: V's scale; dropout: 1 / (1 - p)
         if constexpr (F8) num = p.v_scale[(long)b * p.Hkv + hk];
+        if constexpr (DROP) num = p.drop.inv_keep;
         // block-sparse: a row that saw no visible key keeps m_ref = -inf (its l holds only the
         // clamped polynomial exp2 of -inf): O = 0 and LSE = -inf
         const bool any = SPARSE ? (l > 0.f && m_ref != -INFINITY) : l > 0.f;
@@ -596,9 +631,10 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   const long long num_work = (long long)num_mblk * a.Hq * a.B;
   if (num_work > (1ll << 31) - 1) return cudaErrorInvalidValue;
   Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, a.scale * kLog2e, a.status, num_mblk, (int)num_work,
-           nullptr, nullptr, nullptr, (a.Nq + kBM - 1) / kBM, (a.Nk + kBN - 1) / kBN, a.block_mask};
-  if (a.block_mask) {
-    auto kern = fwd_sm100_kernel<T, D, CAUSAL, false, true>;
+           nullptr, nullptr, nullptr, (a.Nq + kBM - 1) / kBM, (a.Nk + kBN - 1) / kBN, a.block_mask,
+           Dropout{a.drop_thr, a.drop_inv_keep, a.seed_lo, a.seed_hi, a.drop_offset}};
+  if (a.drop_p > 0.f) {
+    auto kern = fwd_sm100_kernel<T, D, CAUSAL, false, false, true>;
     const int smem = Smem<D, false>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -606,7 +642,16 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
     kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mo, p);
     return cudaGetLastError();
   }
-  auto kern = fwd_sm100_kernel<T, D, CAUSAL, false, false>;
+  if (a.block_mask) {
+    auto kern = fwd_sm100_kernel<T, D, CAUSAL, false, true, false>;
+    const int smem = Smem<D, false>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)std::min<long long>(num_work, device_sm_count());
+    kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mo, p);
+    return cudaGetLastError();
+  }
+  auto kern = fwd_sm100_kernel<T, D, CAUSAL, false, false, false>;
   const int smem = Smem<D, false>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -638,8 +683,8 @@ cudaError_t launch_f8(const Fp8AttnArgs& a, cudaStream_t s) {
   if (num_work > (1ll << 31) - 1) return cudaErrorInvalidValue;
   const float sl2 = a.scale * kLog2e / (a.rotated ? (float)D : 1.f);
   Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, sl2, a.status, num_mblk, (int)num_work,
-           a.q_scale, a.k_scale, a.v_scale, (a.Nq + kBM - 1) / kBM, (a.Nk + kBN - 1) / kBN, nullptr};
-  auto kern = fwd_sm100_kernel<T, D, CAUSAL, true, false>;
+           a.q_scale, a.k_scale, a.v_scale, (a.Nq + kBM - 1) / kBM, (a.Nk + kBN - 1) / kBN, nullptr, Dropout{}};
+  auto kern = fwd_sm100_kernel<T, D, CAUSAL, true, false, false>;
   const int smem = Smem<D, true>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

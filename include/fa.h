@@ -186,6 +186,27 @@ fa_status fa_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
                             int num_splits, fa_dtype dt, fa_stream_t stream);
 
 /*
+ * Dropout ("FlashAttention 심층 분석", section 2: dropout is one of the fused steps;
+ * section 4: the backward pass regenerates what it needs).  The mask comes from
+ * Philox4x32-10 (Salmon et al., SC 2011): one call per 2 x 2 block of (query i,
+ * key j) of head (b, h), counter (j >> 1, i >> 1, b * Hq + h, offset), key =
+ * (seed & 0xffffffff, seed >> 32); element (i, j) takes word 2 (i & 1) + (j & 1)
+ * and is kept iff that word >= floor(p_drop * 2^32) (p_drop as passed, in
+ * [0, 1); FA_ERR_INVALID otherwise).  The forward computes
+ * O = (P * M / (1 - p_drop)) V and the LSE of the undropped scores; the
+ * backward (same seed, offset and p_drop) regenerates M and returns the
+ * gradients of sum(dO * O) for that forward.  p_drop = 0 gives fa_fwd /
+ * fa_bwd.  Otherwise as fa_fwd / fa_bwd (layouts, GQA, alignment, workspace).
+ */
+fa_status fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                         int Nq, int Nk, int d, int causal, float scale, float p_drop, unsigned long long seed,
+                         uint32_t offset, fa_dtype dt, fa_stream_t stream);
+fa_status fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                         const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv,
+                         int Nq, int Nk, int d, int causal, float scale, float p_drop, unsigned long long seed,
+                         uint32_t offset, fa_dtype dt, fa_stream_t stream);
+
+/*
  * Block-sparse forward ("FlashAttention-2 (KO)", FA-1 results: the IO-aware
  * kernel extended with a block-sparse pattern).  block_mask: device uint8
  * [B, Hq, ceil(Nq / 128), ceil(Nk / 128)]; entry (b, h, I, J) nonzero means

@@ -167,3 +167,20 @@ def test_blocksparse_rejects_bad_arguments(lib):
     bad = list(base)
     bad[0] = FAKE + 2
     assert lib.fa_fwd_blocksparse(*bad) == -3
+
+
+def test_dropout_rejects_bad_arguments(lib):
+    # q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, p, seed, offset, dt, stream
+    base = [FAKE] * 5 + [1, 4, 2, 8, 8, 128, 0, 0.1, 0.25, 7, 0, 1, None]
+    for p in (1.0, -0.1, float("nan")):
+        bad = list(base)
+        bad[13] = p
+        assert lib.fa_fwd_dropout(*bad) == -1
+    bad = list(base)
+    bad[10] = 96
+    assert lib.fa_fwd_dropout(*bad) == -2
+    bwd = [FAKE] * 10 + [1, 4, 2, 8, 8, 128, 0, 0.1, 1.5, 7, 0, 1, None]
+    assert lib.fa_bwd_dropout(*bwd) == -1
+    bwd[18] = 0.2
+    bwd[9] = None  # workspace
+    assert lib.fa_bwd_dropout(*bwd) == -1
