@@ -274,6 +274,7 @@ def run_ours(args):
                                            peaks_kind)
     sparse = None if args.no_sparse else run_blocksparse(args, torch, fa, _lib, workloads, w, q, k, v, dev, stream,
                                                          world, peaks, peaks_kind)
+    drop = None if args.no_dropout else run_dropout(args, torch, fa, _lib, w, q, k, v, do, dev, stream, world)
     e2e = run_e2e(args, torch, fa, w, q, k, v, do, dev, stream, world, F) if not args.no_e2e else None
 
     cpu = None
@@ -299,6 +300,7 @@ def run_ours(args):
         "decode": decode,
         "fp8": fp8,
         "blocksparse": sparse,
+        "dropout": drop,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -488,6 +490,55 @@ def run_blocksparse(args, torch, fa, _lib, workloads, w, q, k, v, dev, stream, w
             "gpu_launches": K}
 
 
+def run_dropout(args, torch, fa, _lib, w, q, k, v, do, dev, stream, world):
+    """The GQA training step with dropout p = 0.1 (mask regenerated in the backward kernels)."""
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.Nq, w.d
+    p_drop, seed = 0.1, 0x5EED
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, N, device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_workspace_bytes(B, Hq, N), device=dev, dtype=torch.uint8)
+    sh = stream.cuda_stream
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        _lib.fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, N,
+                            d, 1, w.scale, p_drop, seed, 0, _lib.FA_BF16, sh)
+        if ev:
+            ev[1].record(stream)
+        _lib.fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), B, Hq, Hkv, N, N, d, 1,
+                            w.scale, p_drop, seed, 0, _lib.FA_BF16, sh)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    barrier(torch, world)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(torch, world)
+    ms = max_over_ranks(torch, world, t0.elapsed_time(t1)) / K
+    if fa.device_status() != 0:
+        raise RuntimeError("kernel status word set during the dropout section")
+    fwd_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in evs)
+    F = attn_flops(B, Hq, N, N, d, True)
+    return {"workload": f"GQA training step with dropout p={p_drop}: B={B} Hq={Hq} Hkv={Hkv} N={N} d={d} causal bf16",
+            "ms_per_step": round(ms, 4), "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
+            "value": round(world * 3.5 * F / (ms * 1e-3) / 1e12, 1), "unit": "TFLOP/s",
+            "fwd_tflops": round(F / (fwd_ms * 1e-3) / 1e12, 1),
+            "bwd_tflops": round(2.5 * F / (bwd_ms * 1e-3) / 1e12, 1), "gpu_launches": 4 * K}
+
+
 def run_e2e(args, torch, fa, w, q, k, v, do, dev, stream, world, F):
     """Same step through the public Python API with host buffers: pinned H2D of
     q, k, v, dO, forward, backward, D2H of dQ, dK, dV, all inside the timed region."""
@@ -617,6 +668,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode section (profiling runs)")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 forward section (profiling runs)")
     ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse section (profiling runs)")
+    ap.add_argument("--no-dropout", action="store_true", help="skip the dropout section (profiling runs)")
     ap.add_argument("--decode-b", type=int, default=0,
                     help="override B of the decode workload (profiling runs on a smaller case)")
     ap.add_argument("--seq", type=int, default=0,
