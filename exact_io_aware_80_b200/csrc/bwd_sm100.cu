@@ -353,21 +353,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit cc = (query i0 + cc, this key) kept
       if constexpr (DROP) {
+        // lanes 2m and 2m + 1 hold the two keys of one key pair, which share every Philox call:
+        // each lane makes every other call (query pairs) and hands the other key's bits to lane ^ 1
         const uint32_t bh = (uint32_t)(b * p.Hq + hk * G + t / per_head), jp = (uint32_t)key >> 1;
-        const bool kodd = key & 1;
+        const int e = key & 1;  // == lane & 1
 #pragma unroll
         for (int wd = 0; wd < 4; ++wd) {
-          uint32_t m = 0;
+          uint32_t own = 0, other = 0;
 #pragma unroll 1
-          for (int k2 = 0; k2 < 32; k2 += 2) {
+          for (int t2 = 0; t2 < 8; ++t2) {
             // the call of the 2 x 2 block (queries i0 + cc, + 1) x (keys 2 jp, 2 jp + 1)
-            const int cc = 32 * wd + k2;
+            const int cc = 32 * wd + 4 * t2 + 2 * e;
             const uint4 w = philox4x32_10(jp, (uint32_t)(i0 + cc) >> 1, bh, p.drop.offset, p.drop.seed_lo,
                                           p.drop.seed_hi);
-            const uint32_t k0b = (kodd ? w.y : w.x) >= p.drop.thr, k1b = (kodd ? w.w : w.z) >= p.drop.thr;
-            m |= (k0b << k2) | (k1b << (k2 + 1));
+            const uint32_t even = (uint32_t)(w.x >= p.drop.thr) | ((uint32_t)(w.z >= p.drop.thr) << 1);
+            const uint32_t odd = (uint32_t)(w.y >= p.drop.thr) | ((uint32_t)(w.w >= p.drop.thr) << 1);
+            own |= (e ? odd : even) << (cc & 31);
+            other |= (e ? even : odd) << (cc & 31);
           }
-          keep[wd] = m;
+          keep[wd] = own | __shfl_xor_sync(0xffffffffu, other, 1);
         }
       }
       {
@@ -608,20 +612,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit cc = (this query, key kb + cc) kept
       if constexpr (DROP) {
+        // lanes 2m and 2m + 1 hold one query pair: each makes every other call (key pairs) and
+        // hands the other row's bits to lane ^ 1
         const uint32_t bh = (uint32_t)(b * p.Hq + h), rh = (uint32_t)row >> 1;
-        const bool odd = row & 1;
+        const int e = row & 1;  // == lane & 1
 #pragma unroll
         for (int wd = 0; wd < 4; ++wd) {
-          uint32_t m = 0;
+          uint32_t own = 0, other = 0;
 #pragma unroll 1
-          for (int k2 = 0; k2 < 32; k2 += 2) {
-            const int cc = 32 * wd + k2;
+          for (int t2 = 0; t2 < 8; ++t2) {
+            const int cc = 32 * wd + 4 * t2 + 2 * e;
             const uint4 w = philox4x32_10((uint32_t)(kb + cc) >> 1, rh, bh, p.drop.offset, p.drop.seed_lo,
                                           p.drop.seed_hi);
-            const uint32_t k0b = (odd ? w.z : w.x) >= p.drop.thr, k1b = (odd ? w.w : w.y) >= p.drop.thr;
-            m |= (k0b << k2) | (k1b << (k2 + 1));
+            const uint32_t even = (uint32_t)(w.x >= p.drop.thr) | ((uint32_t)(w.y >= p.drop.thr) << 1);
+            const uint32_t odd = (uint32_t)(w.z >= p.drop.thr) | ((uint32_t)(w.w >= p.drop.thr) << 1);
+            own |= (e ? odd : even) << (cc & 31);
+            other |= (e ? even : odd) << (cc & 31);
           }
-          keep[wd] = m;
+          keep[wd] = own | __shfl_xor_sync(0xffffffffu, other, 1);
         }
       }
       write_ds<T, false, DROP>(tbase + lane_off + kColDP, tS, pv, nullptr, ndrow, keep, p.drop.inv_keep);

@@ -484,20 +484,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
         uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit c = (this row, key kbase + c) kept
         if constexpr (DROP) {
+          // lanes 2m and 2m + 1 hold the two rows of one query pair, which share every Philox call:
+          // each lane makes every other call, keeps both rows' bits and hands the other row's to
+          // its partner (lane ^ 1)
           const uint32_t rh = (uint32_t)row >> 1, bh = (uint32_t)(b * p.Hq + h);
-          const bool odd = row & 1;
+          const int e = row & 1;  // == lane & 1
 #pragma unroll
           for (int wd = 0; wd < 4; ++wd) {
-            uint32_t m = 0;
+            uint32_t own = 0, other = 0;
 #pragma unroll 1
-            for (int k2 = 0; k2 < 32; k2 += 2) {
-              // the call of the 2 x 2 block (this row's query pair) x (keys kbase + 32 wd + k2, + 1)
-              const uint4 w = philox4x32_10((uint32_t)(kbase + 32 * wd + k2) >> 1, rh, bh, p.drop.offset,
-                                            p.drop.seed_lo, p.drop.seed_hi);
-              const uint32_t k0b = (odd ? w.z : w.x) >= p.drop.thr, k1b = (odd ? w.w : w.y) >= p.drop.thr;
-              m |= (k0b << k2) | (k1b << (k2 + 1));
+            for (int t2 = 0; t2 < 8; ++t2) {
+              const int c = 32 * wd + 4 * t2 + 2 * e;  // keys kbase + c, + 1: this lane's key pair
+              const uint4 w = philox4x32_10((uint32_t)(kbase + c) >> 1, rh, bh, p.drop.offset, p.drop.seed_lo,
+                                            p.drop.seed_hi);
+              const uint32_t even = (uint32_t)(w.x >= p.drop.thr) | ((uint32_t)(w.y >= p.drop.thr) << 1);
+              const uint32_t odd = (uint32_t)(w.z >= p.drop.thr) | ((uint32_t)(w.w >= p.drop.thr) << 1);
+              own |= (e ? odd : even) << (c & 31);
+              other |= (e ? even : odd) << (c & 31);
             }
-            keep[wd] = m;
+            keep[wd] = own | __shfl_xor_sync(0xffffffffu, other, 1);
           }
         }
         const float2 c2 = make_float2(cj, cj), nm2 = make_float2(-mu, -mu);
