@@ -48,6 +48,7 @@ SIGNATURES = {
     "fa_fp8_v_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I]),
     "fa_fp8_quantize_v": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "fa_lse_merge": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "fa_get_device_status": (_I, [_P]),
     "fa_watchdog_selftest": (_I, [_I, _P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
@@ -173,6 +174,11 @@ def fa_fwd_fp8(q8, q_scale, k8, k_scale, v8t, v_scale, o, lse, B, Hq, Hkv, Nq, N
                stream):
     return _check("fa_fwd_fp8", load().fa_fwd_fp8(q8, q_scale, k8, k_scale, v8t, v_scale, o, lse, B, Hq, Hkv, Nq, Nk,
                                                   d, int(causal), scale, int(rotated), dt, stream))
+
+
+def fa_lse_merge(o_acc, lse_acc, o_part, lse_part, o_out, B, N, H, d, mode, dt, stream):
+    return _check("fa_lse_merge", load().fa_lse_merge(o_acc, lse_acc, o_part, lse_part, o_out, B, N, H, d, mode, dt,
+                                                      stream))
 
 
 def fa_watchdog_selftest(limit_us, stream):

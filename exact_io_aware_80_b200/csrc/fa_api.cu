@@ -182,6 +182,19 @@ fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
   return from_cuda(fa::launch_fwd_sm100(a, static_cast<cudaStream_t>(stream)));
 }
 
+fa_status fa_lse_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
+                       int N, int H, int d, int mode, fa_dtype dt, fa_stream_t stream) {
+  if (!o_acc || !lse_acc || !o_part || !lse_part || (mode == 2 && !o_out)) return FA_ERR_INVALID;
+  if (mode < 0 || mode > 2 || B < 1 || N < 1 || H < 1) return FA_ERR_INVALID;
+  if (dt != FA_FP16 && dt != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(o_acc) || !aligned16(o_part) || (o_out && !aligned16(o_out)) || !aligned4(lse_acc) ||
+      !aligned4(lse_part))
+    return FA_ERR_ALIGN;
+  fa::MergeArgs a{o_acc, lse_acc, o_part, lse_part, o_out, B, N, H, d, mode, dt == FA_BF16 ? 1 : 0};
+  return from_cuda(fa::launch_lse_merge(a, static_cast<cudaStream_t>(stream)));
+}
+
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq) {
   if (B < 1 || Hq < 1 || Nq < 1) return 0;
   return (size_t)B * Hq * Nq * sizeof(float);

@@ -106,6 +106,21 @@ struct Fp8AttnArgs {
   int* status;
 };
 
+// Log-sum-exp merge of a partial attention result (merge.cu): o_acc fp32 [B,N,H,d], lse_acc
+// [B,H,N]; o_part 16-bit [B,N,H,d], lse_part [B,H,N]; mode 0 acc = part, 1 acc = merge,
+// 2 o_out (16-bit [B,N,H,d]) = merge and lse_acc updated.
+struct MergeArgs {
+  float* o_acc;
+  float* lse_acc;
+  const void* o_part;
+  const float* lse_part;
+  void* o_out;
+  int B, N, H, d;
+  int mode;
+  int bf16;
+};
+cudaError_t launch_lse_merge(const MergeArgs& a, cudaStream_t s);
+
 // TMA descriptors (tma.cu).  make_map: 4-D map over a BSHD tensor [B][N][H][D]
 // (innermost d, then head, row, batch); box = 64 columns (128 bytes, 128-byte
 // swizzle) x 1 head x `rows` rows x 1 batch.  Out-of-range rows read as zero.

@@ -274,6 +274,20 @@ fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const
                      int causal, float scale, int rotated, fa_dtype out_dt, fa_stream_t stream);
 
 /*
+ * Log-sum-exp merge of a partial attention result over a disjoint set of keys
+ * into an accumulator ("FlashAttention 심층 분석", "Flash-Decoding": partial
+ * results over key ranges merge by their log-sum-exp); the step that folds each
+ * key/value chunk of a context-parallel ring into the running result.
+ * o_acc fp32 [B, N, H, d] and lse_acc fp32 [B, H, N] (the caller's accumulator);
+ * o_part 16-bit [B, N, H, d] and lse_part [B, H, N] as written by fa_fwd.
+ * mode 0: acc = part; 1: acc = merge(acc, part); 2: o_out 16-bit [B, N, H, d] =
+ * merge(acc, part) and lse_acc = the merged LSE (the last chunk).  A row whose
+ * LSE is -inf in both has O = 0.  o_acc, o_part, o_out 16-byte aligned.
+ */
+fa_status fa_lse_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
+                       int N, int H, int d, int mode, fa_dtype dt, fa_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word that the
  * kernels set when a bounded wait runs out (FA_ERR_TIMEOUT) or a device-side
  * check fails.  Returns FA_OK when no kernel reported an error.

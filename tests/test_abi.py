@@ -184,3 +184,11 @@ def test_dropout_rejects_bad_arguments(lib):
     bwd[18] = 0.2
     bwd[9] = None  # workspace
     assert lib.fa_bwd_dropout(*bwd) == -1
+
+
+def test_lse_merge_rejects_bad_arguments(lib):
+    # o_acc, lse_acc, o_part, lse_part, o_out, B, N, H, d, mode, dt, stream
+    assert lib.fa_lse_merge(FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 2, 128, 2, 1, None) == -1  # mode 2 needs o_out
+    assert lib.fa_lse_merge(FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 2, 128, 3, 1, None) == -1
+    assert lib.fa_lse_merge(FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 2, 96, 1, 1, None) == -2
+    assert lib.fa_lse_merge(FAKE + 4, FAKE, FAKE, FAKE, 0, 1, 8, 2, 128, 1, 1, None) == -3
