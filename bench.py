@@ -275,6 +275,7 @@ def run_ours(args):
     sparse = None if args.no_sparse else run_blocksparse(args, torch, fa, _lib, workloads, w, q, k, v, dev, stream,
                                                          world, peaks, peaks_kind)
     drop = None if args.no_dropout else run_dropout(args, torch, fa, _lib, w, q, k, v, do, dev, stream, world)
+    ringl = None if args.no_ring else run_ring_local(args, torch, w, q, k, v, dev, stream, world)
     e2e = run_e2e(args, torch, fa, w, q, k, v, do, dev, stream, world, F) if not args.no_e2e else None
 
     cpu = None
@@ -301,6 +302,7 @@ def run_ours(args):
         "fp8": fp8,
         "blocksparse": sparse,
         "dropout": drop,
+        "ring_local": ringl,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -539,6 +541,30 @@ def run_dropout(args, torch, fa, _lib, w, q, k, v, do, dev, stream, world):
             "bwd_tflops": round(2.5 * F / (bwd_ms * 1e-3) / 1e12, 1), "gpu_launches": 4 * K}
 
 
+def run_ring_local(args, torch, w, q, k, v, dev, stream, world):
+    """Ring attention forward (context parallelism) for 4 virtual ranks run one after another on this GPU."""
+    from exact_io_aware_80_b200 import ring
+    W = 4
+    for _ in range(args.warmup):
+        ring.ring_attention_fwd_local(q, k, v, W, True, w.scale)
+    K = max(1, args.steps // 2)
+    barrier(torch, world)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(K):
+        ring.ring_attention_fwd_local(q, k, v, W, True, w.scale)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(torch, world)
+    ms = max_over_ranks(torch, world, t0.elapsed_time(t1)) / K
+    F = attn_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, True)
+    return {"workload": f"ring attention forward, {W} virtual ranks on one GPU (no communication), causal: "
+                        f"B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.Nq} d={w.d} bf16",
+            "ms_per_step": round(ms, 4), "value": round(world * F / (ms * 1e-3) / 1e12, 1), "unit": "TFLOP/s",
+            "gpu_launches": K * (W * (W + 1) - 1)}  # W(W+1)/2 forward launches, one merge fewer (rank 0 copies)
+
+
 def run_e2e(args, torch, fa, w, q, k, v, do, dev, stream, world, F):
     """Same step through the public Python API with host buffers: pinned H2D of
     q, k, v, dO, forward, backward, D2H of dQ, dK, dV, all inside the timed region."""
@@ -669,6 +695,7 @@ def main():
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 forward section (profiling runs)")
     ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse section (profiling runs)")
     ap.add_argument("--no-dropout", action="store_true", help="skip the dropout section (profiling runs)")
+    ap.add_argument("--no-ring", action="store_true", help="skip the one-GPU ring-attention section")
     ap.add_argument("--decode-b", type=int, default=0,
                     help="override B of the decode workload (profiling runs on a smaller case)")
     ap.add_argument("--seq", type=int, default=0,
