@@ -72,6 +72,7 @@ __all__ = [
     "eager_softmax_bytes",
     "kv_cache_bytes",
     "brute_force_attention",
+    "attention_bwd_partial",
 ]
 
 
@@ -371,6 +372,38 @@ def decode_combine(O_part, LSE_part):
     wn = np.where(empty, 0.0, w / np.where(empty, 1.0, tot))
     O = np.einsum("bhs,bhsd->bhd", wn, O_part)
     return O[:, None, :, :], lse
+
+
+def attention_bwd_partial(q, k, v, do, lse, dvec, causal: bool, scale: float):
+    """Gradient contributions of one block of keys, given the full rows' LSE and D.
+
+    With P = exp(scale Q K^T - LSE) (the probabilities of the whole row, restricted
+    to these keys), dP = dO V^T and dS = P * (dP - D): dQ_part = scale dS K,
+    dK = scale dS^T Q, dV = P^T dO (dK, dV summed over the query heads of a
+    group).  Summing the parts over a partition of the keys gives the full
+    backward (the chain rule is linear in the keys once LSE and D are fixed);
+    used for context-parallel (ring) attention.  ``lse``, ``dvec``: [B, Hq, Nq].
+    Returns (dQ_part, dK, dV).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    lse, dvec = _f64(lse), _f64(dvec)
+    B, Nq, Nk, Hq, Hkv, d = _check_shapes(q, k, v)
+    G = Hq // Hkv
+    mask = visible_mask(Nq, Nk, causal)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // G
+            S = scores(q[b, :, h, :], k[b, :, hk, :], scale, mask)
+            P = np.exp(S - lse[b, h][:, None])
+            dP = do[b, :, h, :] @ v[b, :, hk, :].T
+            dS = P * (dP - dvec[b, h][:, None])
+            dq[b, :, h, :] = scale * dS @ k[b, :, hk, :]
+            dk[b, :, hk, :] += scale * dS.T @ q[b, :, h, :]
+            dv[b, :, hk, :] += P.T @ do[b, :, h, :]
+    return dq, dk, dv
 
 
 def attention_flops(B: int, Hq: int, Nq: int, Nk: int, d: int, causal: bool, backward: bool = False) -> float:

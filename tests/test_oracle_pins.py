@@ -422,3 +422,30 @@ def _bwd_mutant(kind):
 def test_planted_backward_mistakes_are_caught(kind):
     with pytest.raises(AssertionError):
         check_finite_differences(_bwd_mutant(kind))
+
+
+def test_partial_backward_over_key_chunks_sums_to_the_full_backward():
+    # the backward of a context-parallel ring: per-chunk contributions with the full rows' LSE and D
+    rng = np.random.default_rng(31)
+    q, k, v, do = (rng.standard_normal(s) for s in ((1, 96, 4, 8), (1, 96, 2, 8), (1, 96, 2, 8), (1, 96, 4, 8)))
+    for causal in (False, True):
+        O, L = oracle.attention_fwd(q, k, v, causal, 0.3)
+        D = oracle.bwd_preprocess(O, do)
+        DQ, DK, DV = oracle.attention_bwd(q, k, v, do, causal, 0.3)
+        dq = np.zeros_like(DQ)
+        dk = np.zeros_like(DK)
+        dv = np.zeros_like(DV)
+        n = 32
+        for r in range(3):            # query chunk
+            for c in range(3):        # key chunk
+                if causal and c > r:
+                    continue
+                qs, ks = slice(n * r, n * (r + 1)), slice(n * c, n * (c + 1))
+                a, bb, cc = oracle.attention_bwd_partial(q[:, qs], k[:, ks], v[:, ks], do[:, qs], L[:, :, qs],
+                                                         D[:, :, qs], causal and c == r, 0.3)
+                dq[:, qs] += a
+                dk[:, ks] += bb
+                dv[:, ks] += cc
+        np.testing.assert_allclose(dq, DQ, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dk, DK, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dv, DV, rtol=1e-10, atol=1e-12)
