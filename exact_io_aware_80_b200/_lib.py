@@ -49,6 +49,8 @@ SIGNATURES = {
     "fa_fp8_quantize_v": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "fa_lse_merge": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "fa_accumulate": (_I, [_P, _P, ctypes.c_longlong, _I, _I, _P]),
+    "fa_cast_f32": (_I, [_P, _P, ctypes.c_longlong, _I, _P]),
     "fa_get_device_status": (_I, [_P]),
     "fa_watchdog_selftest": (_I, [_I, _P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
@@ -179,6 +181,14 @@ def fa_fwd_fp8(q8, q_scale, k8, k_scale, v8t, v_scale, o, lse, B, Hq, Hkv, Nq, N
 def fa_lse_merge(o_acc, lse_acc, o_part, lse_part, o_out, B, N, H, d, mode, dt, stream):
     return _check("fa_lse_merge", load().fa_lse_merge(o_acc, lse_acc, o_part, lse_part, o_out, B, N, H, d, mode, dt,
                                                       stream))
+
+
+def fa_accumulate(acc, part, n, init, dt, stream):
+    return _check("fa_accumulate", load().fa_accumulate(acc, part, n, int(init), dt, stream))
+
+
+def fa_cast_f32(acc, out, n, dt, stream):
+    return _check("fa_cast_f32", load().fa_cast_f32(acc, out, n, dt, stream))
 
 
 def fa_watchdog_selftest(limit_us, stream):

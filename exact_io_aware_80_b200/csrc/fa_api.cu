@@ -195,6 +195,21 @@ fa_status fa_lse_merge(float* o_acc, float* lse_acc, const void* o_part, const f
   return from_cuda(fa::launch_lse_merge(a, static_cast<cudaStream_t>(stream)));
 }
 
+fa_status fa_accumulate(float* acc, const void* part, long long n, int init, fa_dtype dt, fa_stream_t stream) {
+  if (!acc || !part || n < 0 || (n & 7)) return FA_ERR_INVALID;
+  if (dt != FA_FP16 && dt != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(acc) || !aligned16(part)) return FA_ERR_ALIGN;
+  return from_cuda(fa::launch_accumulate(acc, part, (long)n, init ? 1 : 0, dt == FA_BF16 ? 1 : 0,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+fa_status fa_cast_f32(const float* acc, void* out, long long n, fa_dtype dt, fa_stream_t stream) {
+  if (!acc || !out || n < 0 || (n & 7)) return FA_ERR_INVALID;
+  if (dt != FA_FP16 && dt != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(acc) || !aligned16(out)) return FA_ERR_ALIGN;
+  return from_cuda(fa::launch_cast(acc, out, (long)n, dt == FA_BF16 ? 1 : 0, static_cast<cudaStream_t>(stream)));
+}
+
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq) {
   if (B < 1 || Hq < 1 || Nq < 1) return 0;
   return (size_t)B * Hq * Nq * sizeof(float);

@@ -120,6 +120,9 @@ struct MergeArgs {
   int bf16;
 };
 cudaError_t launch_lse_merge(const MergeArgs& a, cudaStream_t s);
+// acc fp32[n] = (init ? 0 : acc) + part 16-bit[n]; out 16-bit[n] = acc (n a multiple of 8).
+cudaError_t launch_accumulate(float* acc, const void* part, long n, int init, int bf16, cudaStream_t s);
+cudaError_t launch_cast(const float* acc, void* out, long n, int bf16, cudaStream_t s);
 
 // TMA descriptors (tma.cu).  make_map: 4-D map over a BSHD tensor [B][N][H][D]
 // (innermost d, then head, row, batch); box = 64 columns (128 bytes, 128-byte

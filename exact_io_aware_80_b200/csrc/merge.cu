@@ -8,6 +8,8 @@
 //   L = ln(e^{L_a} + e^{L_p}),  O = e^{L_a - L} O_a + e^{L_p - L} O_p,
 // with -inf for a row that has seen no key (weight 0; both -inf gives O = 0).
 // One warp per (b, row, head); fp32 accumulator, 16-bit partials and output.
+// Also here: the fp32 accumulation of 16-bit gradient partials and the final
+// cast (the backward of the ring sums per-chunk dQ / dK / dV contributions).
 // HBM-bound: per row it moves 4 d (accumulator in) + 2 d (partial) + 4 d
 // (accumulator out) bytes, or 2 d for the final 16-bit output.
 #include <cuda_bf16.h>
@@ -91,7 +93,60 @@ cudaError_t launch_merge_t(const MergeArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// acc = (init ? 0 : acc) + part (16-bit), 8 elements per thread
+template <typename T>
+__global__ void accumulate_kernel(float* __restrict__ acc, const T* __restrict__ part, long n8, int init) {
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const uint4 w = reinterpret_cast<const uint4*>(part)[i];
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+  float4* a4 = reinterpret_cast<float4*>(acc) + 2 * i;
+  float4 lo = init ? make_float4(0.f, 0.f, 0.f, 0.f) : a4[0];
+  float4 hi = init ? make_float4(0.f, 0.f, 0.f, 0.f) : a4[1];
+  const float2 f0 = Elem<T>::unpack(u[0]), f1 = Elem<T>::unpack(u[1]), f2 = Elem<T>::unpack(u[2]),
+               f3 = Elem<T>::unpack(u[3]);
+  lo.x += f0.x; lo.y += f0.y; lo.z += f1.x; lo.w += f1.y;
+  hi.x += f2.x; hi.y += f2.y; hi.z += f3.x; hi.w += f3.y;
+  a4[0] = lo;
+  a4[1] = hi;
+}
+
+// out (16-bit) = acc, 8 elements per thread
+template <typename T>
+__global__ void cast_kernel(const float* __restrict__ acc, T* __restrict__ out, long n8) {
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 lo = reinterpret_cast<const float4*>(acc)[2 * i], hi = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+  reinterpret_cast<uint4*>(out)[i] = make_uint4(Elem<T>::pack(lo.x, lo.y), Elem<T>::pack(lo.z, lo.w),
+                                                Elem<T>::pack(hi.x, hi.y), Elem<T>::pack(hi.z, hi.w));
+}
+
 }  // namespace
+
+cudaError_t launch_accumulate(float* acc, const void* part, long n, int init, int bf16, cudaStream_t s) {
+  const long n8 = n / 8;
+  const long blocks = (n8 + 255) / 256;
+  if (n8 == 0) return cudaSuccess;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  if (bf16)
+    accumulate_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(acc, static_cast<const __nv_bfloat16*>(part), n8,
+                                                                        init);
+  else
+    accumulate_kernel<__half><<<(unsigned)blocks, 256, 0, s>>>(acc, static_cast<const __half*>(part), n8, init);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cast(const float* acc, void* out, long n, int bf16, cudaStream_t s) {
+  const long n8 = n / 8;
+  const long blocks = (n8 + 255) / 256;
+  if (n8 == 0) return cudaSuccess;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  if (bf16)
+    cast_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(acc, static_cast<__nv_bfloat16*>(out), n8);
+  else
+    cast_kernel<__half><<<(unsigned)blocks, 256, 0, s>>>(acc, static_cast<__half*>(out), n8);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_lse_merge(const MergeArgs& a, cudaStream_t s) {
   if (a.bf16) return a.d == 128 ? launch_merge_t<__nv_bfloat16, 128>(a, s) : launch_merge_t<__nv_bfloat16, 64>(a, s);

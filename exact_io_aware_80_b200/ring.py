@@ -1,4 +1,4 @@
-"""Context parallelism: ring attention across ranks (forward).
+"""Context parallelism: ring attention across ranks (forward and backward).
 
 The sequence is split into equal contiguous chunks, one per rank: rank r holds
 queries, keys and values of positions [r n, (r + 1) n).  In step s = 0 .. W-1
@@ -12,11 +12,17 @@ its queries over the whole sequence ("FlashAttention 심층 분석", "Flash-Deco
 attention over disjoint key ranges merges exactly by log-sum-exp; the
 koritips note names ring attention for context lengths past one GPU).
 
-`ring_schedule` is the pure schedule; `ring_attention_fwd` runs it over a
-process group with the library's kernels (or, for host-side tests, with the
-compute functions a caller passes in); `ring_attention_fwd_local` runs the same
-schedule for W virtual ranks on one device, one after another, without
-communication.
+Backward: with the rows' LSE (from the forward) and D = rowsum(dO * O), each
+(query chunk, key chunk) pair contributes exact partial gradients (the dQ and
+dK/dV kernels on that pair); dQ partials are summed in fp32 on the query's
+rank, and the fp32 dK/dV sums of a key chunk travel around the ring with its
+keys and values and reach their owner after one last hop.
+
+`ring_schedule` is the pure schedule; `ring_attention_fwd` / `ring_attention_bwd`
+run it over a process group with the library's kernels (or, for host-side
+tests, with the compute functions a caller passes in); the `_local` variants
+run the same schedule for W virtual ranks on one device, one after another,
+without communication.
 """
 from __future__ import annotations
 
@@ -24,7 +30,8 @@ import math
 
 from . import _lib
 
-__all__ = ["ring_schedule", "ring_attention_fwd", "ring_attention_fwd_local"]
+__all__ = ["ring_schedule", "ring_attention_fwd", "ring_attention_fwd_local", "ring_attention_bwd",
+           "ring_attention_bwd_local"]
 
 
 def ring_schedule(rank: int, world: int, causal: bool):
@@ -73,6 +80,41 @@ class _CudaOps:
         _lib.fa_lse_merge(o_acc.data_ptr(), lse_acc.data_ptr(), o_p.data_ptr(), lse_p.data_ptr(),
                           out.data_ptr() if mode == 2 else 0, B, N, H, d, mode, _dtype(torch, o_p),
                           torch.cuda.current_stream(o_p.device).cuda_stream)
+
+
+    # ----------------------------------------------------------------- backward
+    def preprocess(self, q, k, v, o, do, lse):
+        """D = rowsum(dO * O) of this rank's rows, in a workspace the backward kernels read."""
+        torch = self.torch
+        B, N, Hq, d = q.shape
+        ws = torch.empty(_lib.fa_bwd_workspace_bytes(B, Hq, N), device=q.device, dtype=torch.uint8)
+        _lib.fa_bwd_preprocess(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                               0, 0, 0, ws.data_ptr(), B, Hq, k.shape[2], N, k.shape[1], d, False, self.scale,
+                               _dtype(torch, q), torch.cuda.current_stream(q.device).cuda_stream)
+        return ws
+
+    def partial_bwd(self, q, k, v, o, do, lse, ws, causal):
+        """dQ, dK, dV contributions (16-bit) of one chunk pair, with the rows' LSE and D."""
+        torch = self.torch
+        B, N, Hq, d = q.shape
+        _, Nk, Hkv, _ = k.shape
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+                dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), B, Hq, Hkv, N, Nk, d, causal, self.scale,
+                _dtype(torch, q), torch.cuda.current_stream(q.device).cuda_stream)
+        _lib.fa_bwd_dkdv(*args)
+        _lib.fa_bwd_dq(*args)
+        return dq, dk, dv
+
+    def accumulate(self, acc, part, init):
+        torch = self.torch
+        _lib.fa_accumulate(acc.data_ptr(), part.data_ptr(), part.numel(), init, _dtype(torch, part),
+                           torch.cuda.current_stream(part.device).cuda_stream)
+
+    def cast(self, acc, out):
+        torch = self.torch
+        _lib.fa_cast_f32(acc.data_ptr(), out.data_ptr(), out.numel(), _dtype(torch, out),
+                         torch.cuda.current_stream(out.device).cuda_stream)
 
 
 def _dtype(torch, t):
@@ -165,3 +207,122 @@ def ring_attention_fwd(q, k, v, causal: bool = False, scale: float | None = None
         out.zero_()
         lse.fill_(-math.inf)
     return out, lse
+
+
+def ring_attention_bwd_local(q, k, v, o, do, lse, world: int, causal: bool = False, scale: float | None = None):
+    """The backward ring schedule for `world` virtual ranks on one device (no communication).
+
+    q, o, do [B, N, Hq, d], k/v [B, N, Hkv, d], lse [B, Hq, N] of the whole sequence (N divisible by
+    `world`); returns dQ, dK, dV.
+    """
+    import torch
+    B, N, Hq, d = q.shape
+    if N % world:
+        raise ValueError("sequence length must be a multiple of the number of ranks")
+    n = N // world
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    ops = _CudaOps(torch, scale)
+    sl = [slice(r * n, (r + 1) * n) for r in range(world)]
+    ch = lambda t, r: t[:, sl[r]].contiguous()  # noqa: E731
+    dk_acc = [torch.empty(B, n, k.shape[2], d, device=q.device, dtype=torch.float32) for _ in range(world)]
+    dv_acc = [torch.empty(B, n, k.shape[2], d, device=q.device, dtype=torch.float32) for _ in range(world)]
+    kv_init = [True] * world
+    dq = torch.empty_like(q)
+    for r in range(world):
+        qr, orr, dor = ch(q, r), ch(o, r), ch(do, r)
+        lr = lse[:, :, sl[r]].contiguous()
+        ws = ops.preprocess(qr, ch(k, r), ch(v, r), orr, dor, lr)
+        dq_acc = torch.empty(B, n, Hq, d, device=q.device, dtype=torch.float32)
+        first = True
+        for s_, c, mode in ring_schedule(r, world, causal):
+            if mode == "skip":
+                continue
+            dq_p, dk_p, dv_p = ops.partial_bwd(qr, ch(k, c), ch(v, c), orr, dor, lr, ws, mode == "causal")
+            ops.accumulate(dq_acc, dq_p, first)
+            ops.accumulate(dk_acc[c], dk_p, kv_init[c])
+            ops.accumulate(dv_acc[c], dv_p, kv_init[c])
+            first = False
+            kv_init[c] = False
+        dq_r = torch.empty_like(qr)
+        ops.cast(dq_acc, dq_r)
+        dq[:, sl[r]] = dq_r
+    dk, dv = torch.empty_like(k), torch.empty_like(v)
+    for c in range(world):
+        if kv_init[c]:  # no query attends to this chunk (cannot happen for these schedules)
+            dk[:, sl[c]] = 0
+            dv[:, sl[c]] = 0
+            continue
+        t = torch.empty_like(ch(k, c))
+        ops.cast(dk_acc[c], t)
+        dk[:, sl[c]] = t
+        ops.cast(dv_acc[c], t)
+        dv[:, sl[c]] = t
+    return dq, dk, dv
+
+
+def ring_attention_bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, group=None,
+                       ops=None):
+    """Backward of ring_attention_fwd over a process group: this rank's dQ, dK, dV.
+
+    q, o, do [B, n, Hq, d], k/v [B, n, Hkv, d] and lse [B, Hq, n] are this rank's chunk (lse as returned
+    by ring_attention_fwd: over the whole sequence).  Keys and values travel as in the forward, now with
+    their fp32 dK / dV sums; after the last step the sums take one more hop to their owner.
+    """
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    B, n, Hq, d = q.shape
+    Hkv = k.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    ops = ops or _CudaOps(torch, scale)
+    sched = ring_schedule(rank, world, causal)
+    nxt, prv = (rank + 1) % world, (rank - 1) % world
+    nxt_g = dist.get_global_rank(group, nxt) if group is not None else nxt
+    prv_g = dist.get_global_rank(group, prv) if group is not None else prv
+    ws = ops.preprocess(q, k, v, o, do, lse)
+    dq_acc = torch.empty(B, n, Hq, d, device=q.device, dtype=torch.float32)
+    zeros = lambda: torch.zeros(B, n, Hkv, d, device=q.device, dtype=torch.float32)  # noqa: E731
+    kv = [(k.contiguous(), v.contiguous()), (torch.empty_like(k), torch.empty_like(v))]
+    acc = [(zeros(), zeros()), (zeros(), zeros())]
+
+    def exchange(send, recv):
+        ops_p2p = [dist.P2POp(dist.isend, t, nxt_g, group) for t in send] + \
+                  [dist.P2POp(dist.irecv, t, prv_g, group) for t in recv]
+        return dist.batch_isend_irecv(ops_p2p)
+
+    first = True
+    for s in range(world):
+        cur, nx = s % 2, (s + 1) % 2
+        # keys and values of the next step travel while this step computes
+        reqs = exchange(kv[cur], kv[nx]) if s + 1 < world else []
+        _, c, mode = sched[s]
+        if mode != "skip":
+            dq_p, dk_p, dv_p = ops.partial_bwd(q, kv[cur][0], kv[cur][1], o, do, lse, ws, mode == "causal")
+            ops.accumulate(dq_acc, dq_p, first)
+            ops.accumulate(acc[cur][0], dk_p, False)
+            ops.accumulate(acc[cur][1], dv_p, False)
+            first = False
+        for r_ in reqs:
+            r_.wait()
+        # this chunk's gradient sums move on with it (after this step's contribution)
+        if s + 1 < world:
+            for r_ in exchange(acc[cur], acc[nx]):
+                r_.wait()
+            acc[cur] = (zeros(), zeros())
+    # the sums now held belong to the next rank's chunk: one last hop to their owners
+    last = (world - 1) % 2
+    if world == 1:
+        own = acc[last]
+    else:
+        own = (zeros(), zeros())
+        for r_ in exchange(acc[last], own):
+            r_.wait()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if first:
+        dq.zero_()
+    else:
+        ops.cast(dq_acc, dq)
+    ops.cast(own[0], dk)
+    ops.cast(own[1], dv)
+    return dq, dk, dv

@@ -288,6 +288,16 @@ fa_status fa_lse_merge(float* o_acc, float* lse_acc, const void* o_part, const f
                        int N, int H, int d, int mode, fa_dtype dt, fa_stream_t stream);
 
 /*
+ * Summation of 16-bit partial results in fp32 (the backward of the ring sums the
+ * dQ, dK and dV contributions of every key/value chunk): fa_accumulate sets
+ * acc[i] = (init ? 0 : acc[i]) + part[i] for n elements, fa_cast_f32 writes
+ * out[i] = acc[i] rounded to the 16-bit type.  n a multiple of 8; acc, part and
+ * out 16-byte aligned device pointers.
+ */
+fa_status fa_accumulate(float* acc, const void* part, long long n, int init, fa_dtype dt, fa_stream_t stream);
+fa_status fa_cast_f32(const float* acc, void* out, long long n, fa_dtype dt, fa_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word that the
  * kernels set when a bounded wait runs out (FA_ERR_TIMEOUT) or a device-side
  * check fails.  Returns FA_OK when no kernel reported an error.

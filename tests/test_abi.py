@@ -192,3 +192,11 @@ def test_lse_merge_rejects_bad_arguments(lib):
     assert lib.fa_lse_merge(FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 2, 128, 3, 1, None) == -1
     assert lib.fa_lse_merge(FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 2, 96, 1, 1, None) == -2
     assert lib.fa_lse_merge(FAKE + 4, FAKE, FAKE, FAKE, 0, 1, 8, 2, 128, 1, 1, None) == -3
+
+
+def test_accumulate_and_cast_reject_bad_arguments(lib):
+    assert lib.fa_accumulate(FAKE, FAKE, 12, 1, 1, None) == -1      # n not a multiple of 8
+    assert lib.fa_accumulate(0, FAKE, 16, 1, 1, None) == -1
+    assert lib.fa_accumulate(FAKE + 4, FAKE, 16, 1, 1, None) == -3
+    assert lib.fa_cast_f32(FAKE, FAKE, 16, 5, None) == -2
+    assert lib.fa_cast_f32(FAKE, FAKE + 2, 16, 1, None) == -3

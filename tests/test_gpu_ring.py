@@ -1,7 +1,8 @@
 """Ring attention on one GPU: the ring schedule for W virtual ranks run one
 after another (no communication) with the library's forward and log-sum-exp
 merge kernels must give attention over the whole sequence (oracle): O max-abs
-<= 1e-2, LSE <= 1e-3."""
+<= 1e-2, LSE <= 1e-3; the backward schedule (per-chunk dQ / dK / dV kernels
+summed in fp32) must give the full backward: relative L2 <= 2e-2."""
 import math
 
 import numpy as np
@@ -57,3 +58,20 @@ def test_merge_of_key_halves(fa):
                                 1 / 8)
     assert np.max(np.abs(out.float().cpu().numpy() - O)) <= 1e-2
     assert np.max(np.abs(lse.cpu().numpy() - L)) <= 1e-3
+
+
+@pytest.mark.parametrize("world,causal", [(1, True), (2, False), (4, True)])
+def test_local_ring_backward_is_the_full_backward(fa, world, causal):
+    from exact_io_aware_80_b200 import ring
+    N, d = 160 * world, 128
+    q, k, v, do = workloads.make_inputs(1, 4, 2, N, N, d, torch.bfloat16, seed_base=9200 + world, with_do=True)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, lse = ring.ring_attention_fwd_local(qd, kd, vd, world, causal)
+    dq, dk, dv = ring.ring_attention_bwd_local(qd, kd, vd, o, dod, lse, world, causal)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    DQ, DK, DV = oracle.attention_bwd(q.float().numpy(), k.float().numpy(), v.float().numpy(), do.float().numpy(),
+                                      causal, 1 / math.sqrt(d))
+    for g, G in ((dq, DQ), (dk, DK), (dv, DV)):
+        gg = g.float().cpu().numpy()
+        assert np.linalg.norm(gg - G) / np.linalg.norm(G) <= 2e-2

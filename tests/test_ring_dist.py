@@ -59,6 +59,82 @@ class OracleOps:
             out.copy_(o_acc)
 
 
+class OracleBwdOps:
+    """The backward's compute from the oracle: D, per-chunk-pair partial gradients, fp32 sums."""
+
+    def __init__(self, scale):
+        self.scale = scale
+
+    def preprocess(self, q, k, v, o, do, lse):
+        import oracle
+        return torch.from_numpy(oracle.bwd_preprocess(o.numpy(), do.numpy()))
+
+    def partial_bwd(self, q, k, v, o, do, lse, dvec, causal):
+        import oracle
+        parts = oracle.attention_bwd_partial(q.numpy(), k.numpy(), v.numpy(), do.numpy(), lse.numpy(), dvec.numpy(),
+                                             causal, self.scale)
+        return tuple(torch.from_numpy(x) for x in parts)
+
+    def accumulate(self, acc, part, init):
+        if init:
+            acc.copy_(part)
+        else:
+            acc.add_(part)
+
+    def cast(self, acc, out):
+        out.copy_(acc)
+
+
+def _bwd_rank_main(rank, world, port, causal, out):
+    import torch.distributed as dist
+
+    import oracle
+    from exact_io_aware_80_b200 import ring
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        q, k, v, do = _bwd_inputs(world)
+        O, L = oracle.attention_fwd(q.numpy(), k.numpy(), v.numpy(), causal, 0.25)
+        n = q.shape[1] // world
+        sl = slice(rank * n, (rank + 1) * n)
+        c = lambda t: t[:, sl].contiguous()  # noqa: E731
+        dq, dk, dv = ring.ring_attention_bwd(c(q), c(k), c(v), c(torch.from_numpy(O)), c(do),
+                                             torch.from_numpy(L)[:, :, sl].contiguous(), causal=causal, scale=0.25,
+                                             ops=OracleBwdOps(0.25))
+        out[rank] = (dq.numpy(), dk.numpy(), dv.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def _bwd_inputs(world):
+    g = torch.Generator().manual_seed(12)
+    B, N, Hq, Hkv, d = 1, 40 * world, 4, 2, 8
+    return (torch.randn(B, N, Hq, d, generator=g, dtype=torch.float64),
+            torch.randn(B, N, Hkv, d, generator=g, dtype=torch.float64),
+            torch.randn(B, N, Hkv, d, generator=g, dtype=torch.float64),
+            torch.randn(B, N, Hq, d, generator=g, dtype=torch.float64))
+
+
+@pytest.mark.parametrize("world,causal", [(1, True), (2, False), (2, True), (3, True)])
+def test_ring_backward_over_gloo_ranks_is_the_full_backward(world, causal):
+    import torch.multiprocessing as mp
+
+    import oracle
+    port = _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_bwd_rank_main, args=(world, port, causal, out), nprocs=world, join=True)
+    q, k, v, do = _bwd_inputs(world)
+    DQ, DK, DV = oracle.attention_bwd(q.numpy(), k.numpy(), v.numpy(), do.numpy(), causal, 0.25)
+    n = q.shape[1] // world
+    for r in range(world):
+        dq, dk, dv = out[r]
+        sl = slice(r * n, (r + 1) * n)
+        np.testing.assert_allclose(dq, DQ[:, sl], rtol=0, atol=1e-6)
+        np.testing.assert_allclose(dk, DK[:, sl], rtol=0, atol=1e-6)
+        np.testing.assert_allclose(dv, DV[:, sl], rtol=0, atol=1e-6)
+
+
 def _rank_main(rank, world, port, causal, out):
     import torch.distributed as dist
 
