@@ -19,7 +19,8 @@ def lib():
 
 
 def declared_functions():
-    src = open(HEADER).read()
+    with open(HEADER) as fh:
+        src = fh.read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(fa_\w+)\s*\(", src, flags=re.M)))
 

@@ -45,7 +45,7 @@ def _rank_main(rank, world, port, out):
 def test_two_gloo_ranks_take_the_max_and_scale_weakly():
     import torch.multiprocessing as mp
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
     assert out[0] == out[1]

@@ -23,7 +23,9 @@ def rnd(shape, seed):
 
 
 def test_philox_known_answers():
-    for vec in json.load(open(GOLDEN))["vectors"]:
+    with open(GOLDEN) as fh:
+        vectors = json.load(fh)["vectors"]
+    for vec in vectors:
         c = [int(x, 16) for x in vec["counter"]]
         k = [int(x, 16) for x in vec["key"]]
         out = dr.philox4x32(*[np.array([x]) for x in c], k[0], k[1])

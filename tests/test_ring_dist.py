@@ -121,7 +121,7 @@ def test_ring_backward_over_gloo_ranks_is_the_full_backward(world, causal):
 
     import oracle
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_bwd_rank_main, args=(world, port, causal, out), nprocs=world, join=True)
     q, k, v, do = _bwd_inputs(world)
@@ -162,7 +162,7 @@ def test_ring_over_gloo_ranks_is_exact_attention(world, causal):
 
     import oracle
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_rank_main, args=(world, port, causal, out), nprocs=world, join=True)
     g = torch.Generator().manual_seed(11)
