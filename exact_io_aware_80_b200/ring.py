@@ -1,28 +1,32 @@
 """Context parallelism: ring attention across ranks (forward and backward).
 
-The sequence is split into equal contiguous chunks, one per rank: rank r holds
-queries, keys and values of positions [r n, (r + 1) n).  In step s = 0 .. W-1
-rank r holds the key/value chunk c = (r - s) mod W, attends its queries to it
-(causal: c < r all keys, c == r the causal diagonal, c > r nothing) with the
-16-bit forward kernel, and folds the partial (O, LSE) into an fp32 accumulator
-with the log-sum-exp merge kernel; meanwhile it sends its chunk to rank r + 1
-and receives the next from rank r - 1 (point-to-point sends over the process
-group, NCCL between GPUs).  After W steps every rank holds exact attention of
-its queries over the whole sequence ("FlashAttention 심층 분석", "Flash-Decoding":
-attention over disjoint key ranges merges exactly by log-sum-exp; the
-koritips note names ring attention for context lengths past one GPU).
+The sequence is split into parts: W equal contiguous parts, rank r owning part
+r ("contiguous"), or 2W parts with rank r owning parts r and 2W - 1 - r
+("zigzag", which gives every rank the same causal work).  A rank holds the
+queries, keys and values of its parts, concatenated in that order.  In step
+s = 0 .. W-1 rank r holds the keys and values of rank c = (r - s) mod W and
+attends each of its query parts a to each held key part b (causal: b < a all
+keys, b == a the causal diagonal, b > a nothing) with the 16-bit forward
+kernel, folding each partial (O, LSE) into that query part's fp32 accumulator
+with the log-sum-exp merge kernel; meanwhile it sends the keys and values it
+holds to rank r + 1 and receives the next from rank r - 1 (point-to-point sends
+over the process group, NCCL between GPUs).  After W steps every rank holds
+exact attention of its queries over the whole sequence ("FlashAttention 심층
+분석", "Flash-Decoding": attention over disjoint key ranges merges exactly by
+log-sum-exp; the koritips note names ring attention for context lengths past
+one GPU).
 
 Backward: with the rows' LSE (from the forward) and D = rowsum(dO * O), each
-(query chunk, key chunk) pair contributes exact partial gradients (the dQ and
+(query part, key part) pair contributes exact partial gradients (the dQ and
 dK/dV kernels on that pair); dQ partials are summed in fp32 on the query's
-rank, and the fp32 dK/dV sums of a key chunk travel around the ring with its
-keys and values and reach their owner after one last hop.
+rank, and the fp32 dK/dV sums of the held key parts travel around the ring
+with their keys and values and reach their owner after one last hop.
 
 `ring_schedule` is the pure schedule; `ring_attention_fwd` / `ring_attention_bwd`
 run it over a process group with the library's kernels (or, for host-side
 tests, with the compute functions a caller passes in); the `_local` variants
 run the same schedule for W virtual ranks on one device, one after another,
-without communication.
+without communication, taking and returning whole-sequence tensors.
 """
 from __future__ import annotations
 
@@ -30,24 +34,40 @@ import math
 
 from . import _lib
 
-__all__ = ["ring_schedule", "ring_attention_fwd", "ring_attention_fwd_local", "ring_attention_bwd",
-           "ring_attention_bwd_local"]
+__all__ = ["owned_parts", "num_parts", "ring_schedule", "ring_attention_fwd", "ring_attention_fwd_local",
+           "ring_attention_bwd", "ring_attention_bwd_local"]
+
+LAYOUTS = ("contiguous", "zigzag")
 
 
-def ring_schedule(rank: int, world: int, causal: bool):
-    """[(step, chunk, mode)] for one rank; mode "full", "causal" (diagonal chunk) or "skip"."""
+def num_parts(world: int, layout: str) -> int:
+    """Number of sequence parts: W (contiguous) or 2W (zigzag)."""
+    if layout not in LAYOUTS:
+        raise ValueError(f"layout must be one of {LAYOUTS}")
+    return world if layout == "contiguous" else 2 * world
+
+
+def owned_parts(rank: int, world: int, layout: str = "contiguous"):
+    """Global part indices rank `rank` holds, in the order its local tensors concatenate them."""
     if not 0 <= rank < world:
         raise ValueError("rank out of range")
+    return [rank] if num_parts(world, layout) == world else [rank, 2 * world - 1 - rank]
+
+
+def ring_schedule(rank: int, world: int, causal: bool, layout: str = "contiguous"):
+    """[(step, held rank, [(own part idx, held part idx, mode)])]; mode "full" or "causal", skipped pairs left out."""
+    mine = owned_parts(rank, world, layout)
     out = []
     for s in range(world):
         c = (rank - s) % world
-        if not causal or c < rank:
-            mode = "full"
-        elif c == rank:
-            mode = "causal"
-        else:
-            mode = "skip"
-        out.append((s, c, mode))
+        pairs = []
+        for ia, a in enumerate(mine):
+            for ib, b in enumerate(owned_parts(c, world, layout)):
+                if not causal or b < a:
+                    pairs.append((ia, ib, "full"))
+                elif b == a:
+                    pairs.append((ia, ib, "causal"))
+        out.append((s, c, pairs))
     return out
 
 
@@ -121,208 +141,272 @@ def _dtype(torch, t):
     return _lib.FA_BF16 if t.dtype == torch.bfloat16 else _lib.FA_FP16
 
 
-def _run_schedule(sched, q, get_kv, ops, out, lse, o_acc, torch):
-    """Partial attention per non-skipped step, merged in step order into (o_acc, lse) -> out."""
-    work = [(s, c, m) for s, c, m in sched if m != "skip"]
-    first = True
-    for i, (s, c, mode) in enumerate(work):
-        k, v = get_kv(s)
-        part = ops.partial(q, k, v, mode == "causal")
-        ops.merge((o_acc, lse, out, first), part, i == len(work) - 1)
-        first = False
-    return out, lse
+def _dtype(torch, t):
+    return _lib.FA_BF16 if t.dtype == torch.bfloat16 else _lib.FA_FP16
 
 
-def ring_attention_fwd_local(q, k, v, world: int, causal: bool = False, scale: float | None = None):
+def _split(t, P):
+    """P contiguous parts of t along the sequence axis (dim 1)."""
+    n = t.shape[1] // P
+    return [t[:, i * n:(i + 1) * n].contiguous() for i in range(P)]
+
+
+def _split_lse(t, P):
+    n = t.shape[2] // P
+    return [t[:, :, i * n:(i + 1) * n].contiguous() for i in range(P)]
+
+
+def _fwd_rank(torch, ops, sched, q_parts, held_kv):
+    """Forward of one rank: partials of every scheduled (query part, key part) pair merged per query part.
+
+    held_kv(step) -> list of (k, v) parts held at that step.  Returns lists of O and LSE per own part.
+    """
+    P = len(q_parts)
+    remaining = [0] * P
+    for _, _, pairs in sched:
+        for ia, _, _ in pairs:
+            remaining[ia] += 1
+    B, n, Hq, d = q_parts[0].shape
+    outs = [torch.empty_like(qp) for qp in q_parts]
+    lses = [torch.empty(B, Hq, n, device=qp.device, dtype=torch.float32) for qp in q_parts]
+    accs = [torch.empty(B, n, Hq, d, device=qp.device, dtype=torch.float32) for qp in q_parts]
+    first = [True] * P
+    for s, _, pairs in sched:
+        kv = held_kv(s)
+        for ia, ib, mode in pairs:
+            part = ops.partial(q_parts[ia], kv[ib][0], kv[ib][1], mode == "causal")
+            remaining[ia] -= 1
+            ops.merge((accs[ia], lses[ia], outs[ia], first[ia]), part, remaining[ia] == 0)
+            first[ia] = False
+    for ia in range(P):
+        if first[ia]:  # no key part attends to these queries (cannot happen for these schedules)
+            outs[ia].zero_()
+            lses[ia].fill_(-math.inf)
+    return outs, lses
+
+
+def ring_attention_fwd_local(q, k, v, world: int, causal: bool = False, scale: float | None = None,
+                             layout: str = "contiguous"):
     """The ring schedule for `world` virtual ranks on one device (no communication).
 
-    q [B, N, Hq, d], k/v [B, N, Hkv, d] with N divisible by `world`; returns O, LSE of the whole sequence.
+    q [B, N, Hq, d], k/v [B, N, Hkv, d] of the whole sequence, N divisible by the number of parts;
+    returns O, LSE of the whole sequence.
     """
     import torch
     B, N, Hq, d = q.shape
-    if N % world:
-        raise ValueError("sequence length must be a multiple of the number of ranks")
-    n = N // world
+    NP = num_parts(world, layout)
+    if N % NP:
+        raise ValueError("sequence length must be a multiple of the number of parts")
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     ops = _CudaOps(torch, scale)
+    qg, kg, vg = _split(q, NP), _split(k, NP), _split(v, NP)
     out = torch.empty_like(q)
     lse = torch.empty(B, Hq, N, device=q.device, dtype=torch.float32)
+    n = N // NP
     for r in range(world):
-        qr = q[:, r * n:(r + 1) * n].contiguous()
-        o_acc = torch.empty(B, n, Hq, d, device=q.device, dtype=torch.float32)
-        lse_r = torch.empty(B, Hq, n, device=q.device, dtype=torch.float32)
-        out_r = torch.empty_like(qr)
-        chunks = {c: (k[:, c * n:(c + 1) * n].contiguous(), v[:, c * n:(c + 1) * n].contiguous()) for c in range(world)}
-        sched = ring_schedule(r, world, causal)
-        _run_schedule(sched, qr, lambda s: chunks[sched[s][1]], ops, out_r, lse_r, o_acc, torch)
-        out[:, r * n:(r + 1) * n] = out_r
-        lse[:, :, r * n:(r + 1) * n] = lse_r
+        mine = owned_parts(r, world, layout)
+        sched = ring_schedule(r, world, causal, layout)
+        held = lambda s, sched=sched: [(kg[b], vg[b]) for b in owned_parts(sched[s][1], world, layout)]  # noqa: E731
+        outs, lses = _fwd_rank(torch, ops, sched, [qg[a] for a in mine], held)
+        for ia, a in enumerate(mine):
+            out[:, a * n:(a + 1) * n] = outs[ia]
+            lse[:, :, a * n:(a + 1) * n] = lses[ia]
     return out, lse
 
 
-def ring_attention_fwd(q, k, v, causal: bool = False, scale: float | None = None, group=None, ops=None):
-    """Ring attention over a process group; q, k, v are this rank's chunk ([B, n, H, d]).
+def _p2p(dist, group, nxt, prv, send, recv):
+    ops_p2p = [dist.P2POp(dist.isend, t, nxt, group) for t in send] + \
+              [dist.P2POp(dist.irecv, t, prv, group) for t in recv]
+    return dist.batch_isend_irecv(ops_p2p) if ops_p2p else []
+
+
+def _neighbours(dist, group, rank, world):
+    nxt, prv = (rank + 1) % world, (rank - 1) % world
+    if group is not None:
+        nxt, prv = dist.get_global_rank(group, nxt), dist.get_global_rank(group, prv)
+    return nxt, prv
+
+
+def ring_attention_fwd(q, k, v, causal: bool = False, scale: float | None = None, group=None, ops=None,
+                       layout: str = "contiguous"):
+    """Ring attention over a process group; q, k, v are this rank's parts concatenated ([B, n, H, d]).
 
     Returns this rank's O [B, n, Hq, d] and LSE [B, Hq, n].  `ops` (partial, merge) defaults to the
-    library's CUDA kernels; the sends and receives of the K/V chunks overlap the compute of each step.
+    library's CUDA kernels; the sends and receives of the keys and values overlap each step's compute.
     """
     import torch
     import torch.distributed as dist
-    world = dist.get_world_size(group)
-    rank = dist.get_rank(group)
-    B, n, Hq, d = q.shape
-    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    P = len(owned_parts(rank, world, layout))
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
     ops = ops or _CudaOps(torch, scale)
-    acc_dtype = torch.float32
-    out = torch.empty_like(q)
-    lse = torch.empty(B, Hq, n, device=q.device, dtype=torch.float32)
-    o_acc = torch.empty(B, n, Hq, d, device=q.device, dtype=acc_dtype)
-    sched = ring_schedule(rank, world, causal)
-    nxt, prv = (rank + 1) % world, (rank - 1) % world
-    nxt_g = dist.get_global_rank(group, nxt) if group is not None else nxt
-    prv_g = dist.get_global_rank(group, prv) if group is not None else prv
-    cur = (k.contiguous(), v.contiguous())
-    bufs = [cur, (torch.empty_like(cur[0]), torch.empty_like(cur[1]))]
-    # step s computes on bufs[s % 2] while the chunk for step s + 1 travels into bufs[(s + 1) % 2]
-    work = [(s, c, m) for s, c, m in sched if m != "skip"]
-    first = True
-    done = 0
-    for s in range(world):
-        reqs = []
+    sched = ring_schedule(rank, world, causal, layout)
+    nxt, prv = _neighbours(dist, group, rank, world)
+    q_parts = _split(q, P)
+    bufs = [list(zip(_split(k, P), _split(v, P))), [(torch.empty_like(kk), torch.empty_like(vv))
+                                                    for kk, vv in zip(_split(k, P), _split(v, P))]]
+    pending = {}
+
+    def held(s):
+        # the keys and values of step s + 1 start travelling before step s computes
+        for r_ in pending.pop(s, []):
+            r_.wait()
         if s + 1 < world:
             src, dst = bufs[s % 2], bufs[(s + 1) % 2]
-            ops_p2p = [dist.P2POp(dist.isend, src[0], nxt_g, group), dist.P2POp(dist.isend, src[1], nxt_g, group),
-                       dist.P2POp(dist.irecv, dst[0], prv_g, group), dist.P2POp(dist.irecv, dst[1], prv_g, group)]
-            reqs = dist.batch_isend_irecv(ops_p2p)
-        _, c, mode = sched[s]
-        if mode != "skip":
-            kc, vc = bufs[s % 2]
-            part = ops.partial(q, kc, vc, mode == "causal")
-            done += 1
-            ops.merge((o_acc, lse, out, first), part, done == len(work))
-            first = False
-        for r in reqs:
-            r.wait()
-    if not work:  # every key chunk is after this rank's queries (cannot happen for causal rank order)
-        out.zero_()
-        lse.fill_(-math.inf)
-    return out, lse
+            pending[s + 1] = _p2p(dist, group, nxt, prv, [t for kv in src for t in kv], [t for kv in dst for t in kv])
+        return bufs[s % 2]
+
+    outs, lses = _fwd_rank(torch, ops, sched, q_parts, held)
+    for reqs in pending.values():
+        for r_ in reqs:
+            r_.wait()
+    return torch.cat(outs, dim=1), torch.cat(lses, dim=2)
 
 
-def ring_attention_bwd_local(q, k, v, o, do, lse, world: int, causal: bool = False, scale: float | None = None):
+def _bwd_rank(torch, ops, sched, qp, op, dop, lp, held, add_kv_grad):
+    """Backward of one rank: dQ sums per own part; per held key part, add_kv_grad(step, ib, dk, dv)."""
+    P = len(qp)
+    wss = [ops.preprocess(qp[i], qp[i], qp[i], op[i], dop[i], lp[i]) for i in range(P)]
+    B, n, Hq, d = qp[0].shape
+    dq_acc = [torch.empty(B, n, Hq, d, device=qp[0].device, dtype=torch.float32) for _ in range(P)]
+    first = [True] * P
+    for s, _, pairs in sched:
+        kv = held(s)
+        for ia, ib, mode in pairs:
+            dq_p, dk_p, dv_p = ops.partial_bwd(qp[ia], kv[ib][0], kv[ib][1], op[ia], dop[ia], lp[ia], wss[ia],
+                                               mode == "causal")
+            ops.accumulate(dq_acc[ia], dq_p, first[ia])
+            first[ia] = False
+            add_kv_grad(s, ib, dk_p, dv_p)
+    dq = [torch.empty_like(x) for x in qp]
+    for i in range(P):
+        if first[i]:
+            dq[i].zero_()
+        else:
+            ops.cast(dq_acc[i], dq[i])
+    return dq
+
+
+def ring_attention_bwd_local(q, k, v, o, do, lse, world: int, causal: bool = False, scale: float | None = None,
+                             layout: str = "contiguous"):
     """The backward ring schedule for `world` virtual ranks on one device (no communication).
 
-    q, o, do [B, N, Hq, d], k/v [B, N, Hkv, d], lse [B, Hq, N] of the whole sequence (N divisible by
-    `world`); returns dQ, dK, dV.
+    Whole-sequence q, o, do [B, N, Hq, d], k/v [B, N, Hkv, d], lse [B, Hq, N]; returns dQ, dK, dV.
     """
     import torch
     B, N, Hq, d = q.shape
-    if N % world:
-        raise ValueError("sequence length must be a multiple of the number of ranks")
-    n = N // world
+    NP = num_parts(world, layout)
+    if N % NP:
+        raise ValueError("sequence length must be a multiple of the number of parts")
+    n = N // NP
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     ops = _CudaOps(torch, scale)
-    sl = [slice(r * n, (r + 1) * n) for r in range(world)]
-    ch = lambda t, r: t[:, sl[r]].contiguous()  # noqa: E731
-    dk_acc = [torch.empty(B, n, k.shape[2], d, device=q.device, dtype=torch.float32) for _ in range(world)]
-    dv_acc = [torch.empty(B, n, k.shape[2], d, device=q.device, dtype=torch.float32) for _ in range(world)]
-    kv_init = [True] * world
+    qg, kg, vg, og, dog, lg = _split(q, NP), _split(k, NP), _split(v, NP), _split(o, NP), _split(do, NP), \
+        _split_lse(lse, NP)
+    Hkv = k.shape[2]
+    dk_acc = [torch.empty(B, n, Hkv, d, device=q.device, dtype=torch.float32) for _ in range(NP)]
+    dv_acc = [torch.empty(B, n, Hkv, d, device=q.device, dtype=torch.float32) for _ in range(NP)]
+    kv_first = [True] * NP
     dq = torch.empty_like(q)
     for r in range(world):
-        qr, orr, dor = ch(q, r), ch(o, r), ch(do, r)
-        lr = lse[:, :, sl[r]].contiguous()
-        ws = ops.preprocess(qr, ch(k, r), ch(v, r), orr, dor, lr)
-        dq_acc = torch.empty(B, n, Hq, d, device=q.device, dtype=torch.float32)
-        first = True
-        for s_, c, mode in ring_schedule(r, world, causal):
-            if mode == "skip":
-                continue
-            dq_p, dk_p, dv_p = ops.partial_bwd(qr, ch(k, c), ch(v, c), orr, dor, lr, ws, mode == "causal")
-            ops.accumulate(dq_acc, dq_p, first)
-            ops.accumulate(dk_acc[c], dk_p, kv_init[c])
-            ops.accumulate(dv_acc[c], dv_p, kv_init[c])
-            first = False
-            kv_init[c] = False
-        dq_r = torch.empty_like(qr)
-        ops.cast(dq_acc, dq_r)
-        dq[:, sl[r]] = dq_r
+        mine = owned_parts(r, world, layout)
+        sched = ring_schedule(r, world, causal, layout)
+
+        def held(s, sched=sched):
+            return [(kg[b], vg[b]) for b in owned_parts(sched[s][1], world, layout)]
+
+        def add(s, ib, dk_p, dv_p, sched=sched):
+            b = owned_parts(sched[s][1], world, layout)[ib]
+            ops.accumulate(dk_acc[b], dk_p, kv_first[b])
+            ops.accumulate(dv_acc[b], dv_p, kv_first[b])
+            kv_first[b] = False
+
+        dqs = _bwd_rank(torch, ops, sched, [qg[a] for a in mine], [og[a] for a in mine], [dog[a] for a in mine],
+                        [lg[a] for a in mine], held, add)
+        for ia, a in enumerate(mine):
+            dq[:, a * n:(a + 1) * n] = dqs[ia]
     dk, dv = torch.empty_like(k), torch.empty_like(v)
-    for c in range(world):
-        if kv_init[c]:  # no query attends to this chunk (cannot happen for these schedules)
-            dk[:, sl[c]] = 0
-            dv[:, sl[c]] = 0
+    for b in range(NP):
+        t = torch.empty_like(kg[b])
+        if kv_first[b]:
+            t.zero_()
+            dk[:, b * n:(b + 1) * n] = t
+            dv[:, b * n:(b + 1) * n] = t
             continue
-        t = torch.empty_like(ch(k, c))
-        ops.cast(dk_acc[c], t)
-        dk[:, sl[c]] = t
-        ops.cast(dv_acc[c], t)
-        dv[:, sl[c]] = t
+        ops.cast(dk_acc[b], t)
+        dk[:, b * n:(b + 1) * n] = t
+        ops.cast(dv_acc[b], t)
+        dv[:, b * n:(b + 1) * n] = t
     return dq, dk, dv
 
 
 def ring_attention_bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, group=None,
-                       ops=None):
+                       ops=None, layout: str = "contiguous"):
     """Backward of ring_attention_fwd over a process group: this rank's dQ, dK, dV.
 
-    q, o, do [B, n, Hq, d], k/v [B, n, Hkv, d] and lse [B, Hq, n] are this rank's chunk (lse as returned
-    by ring_attention_fwd: over the whole sequence).  Keys and values travel as in the forward, now with
-    their fp32 dK / dV sums; after the last step the sums take one more hop to their owner.
+    q, o, do [B, n, Hq, d], k/v [B, n, Hkv, d] and lse [B, Hq, n] are this rank's parts (lse as returned by
+    ring_attention_fwd: over the whole sequence).  Keys and values travel as in the forward, with the fp32
+    dK / dV sums of their parts; after the last step the sums take one more hop to their owner.
     """
     import torch
     import torch.distributed as dist
-    world = dist.get_world_size(group)
-    rank = dist.get_rank(group)
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    P = len(owned_parts(rank, world, layout))
     B, n, Hq, d = q.shape
     Hkv = k.shape[2]
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     ops = ops or _CudaOps(torch, scale)
-    sched = ring_schedule(rank, world, causal)
-    nxt, prv = (rank + 1) % world, (rank - 1) % world
-    nxt_g = dist.get_global_rank(group, nxt) if group is not None else nxt
-    prv_g = dist.get_global_rank(group, prv) if group is not None else prv
-    ws = ops.preprocess(q, k, v, o, do, lse)
-    dq_acc = torch.empty(B, n, Hq, d, device=q.device, dtype=torch.float32)
-    zeros = lambda: torch.zeros(B, n, Hkv, d, device=q.device, dtype=torch.float32)  # noqa: E731
-    kv = [(k.contiguous(), v.contiguous()), (torch.empty_like(k), torch.empty_like(v))]
-    acc = [(zeros(), zeros()), (zeros(), zeros())]
-
-    def exchange(send, recv):
-        ops_p2p = [dist.P2POp(dist.isend, t, nxt_g, group) for t in send] + \
-                  [dist.P2POp(dist.irecv, t, prv_g, group) for t in recv]
-        return dist.batch_isend_irecv(ops_p2p)
-
-    first = True
-    for s in range(world):
-        cur, nx = s % 2, (s + 1) % 2
-        # keys and values of the next step travel while this step computes
-        reqs = exchange(kv[cur], kv[nx]) if s + 1 < world else []
-        _, c, mode = sched[s]
-        if mode != "skip":
-            dq_p, dk_p, dv_p = ops.partial_bwd(q, kv[cur][0], kv[cur][1], o, do, lse, ws, mode == "causal")
-            ops.accumulate(dq_acc, dq_p, first)
-            ops.accumulate(acc[cur][0], dk_p, False)
-            ops.accumulate(acc[cur][1], dv_p, False)
-            first = False
-        for r_ in reqs:
+    sched = ring_schedule(rank, world, causal, layout)
+    nxt, prv = _neighbours(dist, group, rank, world)
+    np_ = n // P
+    zeros = lambda: torch.zeros(B, np_, Hkv, d, device=q.device, dtype=torch.float32)  # noqa: E731
+    kv = [list(zip(_split(k, P), _split(v, P))), [(torch.empty_like(kk), torch.empty_like(vv))
+                                                  for kk, vv in zip(_split(k, P), _split(v, P))]]
+    acc = [[(zeros(), zeros()) for _ in range(P)], [(zeros(), zeros()) for _ in range(P)]]
+    qp, op, dop, lp = _split(q, P), _split(o, P), _split(do, P), _split_lse(lse, P)
+    wss = [ops.preprocess(qp[i], qp[i], qp[i], op[i], dop[i], lp[i]) for i in range(P)]
+    dq_acc = [torch.empty(B, np_, Hq, d, device=q.device, dtype=torch.float32) for _ in range(P)]
+    first = [True] * P
+    pending = []
+    for s, _, pairs in sched:
+        for r_ in pending:
             r_.wait()
-        # this chunk's gradient sums move on with it (after this step's contribution)
+        pending = []
+        cur_kv = kv[s % 2]
+        if s + 1 < world:  # the keys and values of the next step travel while this step computes
+            pending = _p2p(dist, group, nxt, prv, [t for x in cur_kv for t in x], [t for x in kv[(s + 1) % 2] for t in x])
+        for ia, ib, mode in pairs:
+            dq_p, dk_p, dv_p = ops.partial_bwd(qp[ia], cur_kv[ib][0], cur_kv[ib][1], op[ia], dop[ia], lp[ia],
+                                               wss[ia], mode == "causal")
+            ops.accumulate(dq_acc[ia], dq_p, first[ia])
+            first[ia] = False
+            ops.accumulate(acc[s % 2][ib][0], dk_p, False)
+            ops.accumulate(acc[s % 2][ib][1], dv_p, False)
         if s + 1 < world:
-            for r_ in exchange(acc[cur], acc[nx]):
+            # the held parts' gradient sums move on with them, after this step's contributions
+            for r_ in _p2p(dist, group, nxt, prv, [t for x in acc[s % 2] for t in x],
+                           [t for x in acc[(s + 1) % 2] for t in x]):
                 r_.wait()
-            acc[cur] = (zeros(), zeros())
-    # the sums now held belong to the next rank's chunk: one last hop to their owners
-    last = (world - 1) % 2
+            acc[s % 2] = [(zeros(), zeros()) for _ in range(P)]
+    for r_ in pending:
+        r_.wait()
+    # the sums now held belong to the next rank's parts: one last hop to their owners
+    last = acc[(world - 1) % 2]
     if world == 1:
-        own = acc[last]
+        own = last
     else:
-        own = (zeros(), zeros())
-        for r_ in exchange(acc[last], own):
+        own = [(zeros(), zeros()) for _ in range(P)]
+        for r_ in _p2p(dist, group, nxt, prv, [t for x in last for t in x], [t for x in own for t in x]):
             r_.wait()
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    if first:
-        dq.zero_()
-    else:
-        ops.cast(dq_acc, dq)
-    ops.cast(own[0], dk)
-    ops.cast(own[1], dv)
-    return dq, dk, dv
+    dq_parts = [torch.empty_like(x) for x in qp]
+    for i in range(P):
+        if first[i]:
+            dq_parts[i].zero_()
+        else:
+            ops.cast(dq_acc[i], dq_parts[i])
+    dk_parts = [torch.empty(B, np_, Hkv, d, device=q.device, dtype=k.dtype) for _ in range(P)]
+    dv_parts = [torch.empty(B, np_, Hkv, d, device=q.device, dtype=v.dtype) for _ in range(P)]
+    for i in range(P):
+        ops.cast(own[i][0], dk_parts[i])
+        ops.cast(own[i][1], dv_parts[i])
+    return torch.cat(dq_parts, dim=1), torch.cat(dk_parts, dim=1), torch.cat(dv_parts, dim=1)

@@ -25,13 +25,17 @@ def fa():
     return m
 
 
-@pytest.mark.parametrize("world,causal,d,dt", [(1, True, 128, torch.bfloat16), (2, False, 128, torch.bfloat16),
-                                               (4, True, 128, torch.bfloat16), (3, True, 64, torch.float16)])
-def test_local_ring_is_exact_attention(fa, world, causal, d, dt):
+@pytest.mark.parametrize("world,causal,d,dt,layout", [(1, True, 128, torch.bfloat16, "contiguous"),
+                                                      (2, False, 128, torch.bfloat16, "contiguous"),
+                                                      (4, True, 128, torch.bfloat16, "contiguous"),
+                                                      (3, True, 64, torch.float16, "contiguous"),
+                                                      (2, True, 128, torch.bfloat16, "zigzag"),
+                                                      (4, True, 64, torch.float16, "zigzag")])
+def test_local_ring_is_exact_attention(fa, world, causal, d, dt, layout):
     from exact_io_aware_80_b200 import ring
     N = 192 * world
     q, k, v = workloads.make_inputs(1, 4, 2, N, N, d, dt, seed_base=9000 + world)
-    o, lse = ring.ring_attention_fwd_local(q.cuda(), k.cuda(), v.cuda(), world, causal)
+    o, lse = ring.ring_attention_fwd_local(q.cuda(), k.cuda(), v.cuda(), world, causal, layout=layout)
     torch.cuda.synchronize()
     assert fa.device_status() == 0
     O, L = oracle.attention_fwd(q.float().numpy(), k.float().numpy(), v.float().numpy(), causal, 1 / math.sqrt(d))
@@ -60,14 +64,15 @@ def test_merge_of_key_halves(fa):
     assert np.max(np.abs(lse.cpu().numpy() - L)) <= 1e-3
 
 
-@pytest.mark.parametrize("world,causal", [(1, True), (2, False), (4, True)])
-def test_local_ring_backward_is_the_full_backward(fa, world, causal):
+@pytest.mark.parametrize("world,causal,layout", [(1, True, "contiguous"), (2, False, "contiguous"),
+                                                 (4, True, "contiguous"), (2, True, "zigzag"), (3, True, "zigzag")])
+def test_local_ring_backward_is_the_full_backward(fa, world, causal, layout):
     from exact_io_aware_80_b200 import ring
     N, d = 160 * world, 128
     q, k, v, do = workloads.make_inputs(1, 4, 2, N, N, d, torch.bfloat16, seed_base=9200 + world, with_do=True)
     qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
-    o, lse = ring.ring_attention_fwd_local(qd, kd, vd, world, causal)
-    dq, dk, dv = ring.ring_attention_bwd_local(qd, kd, vd, o, dod, lse, world, causal)
+    o, lse = ring.ring_attention_fwd_local(qd, kd, vd, world, causal, layout=layout)
+    dq, dk, dv = ring.ring_attention_bwd_local(qd, kd, vd, o, dod, lse, world, causal, layout=layout)
     torch.cuda.synchronize()
     assert fa.device_status() == 0
     DQ, DK, DV = oracle.attention_bwd(q.float().numpy(), k.float().numpy(), v.float().numpy(), do.float().numpy(),

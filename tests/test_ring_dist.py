@@ -85,7 +85,7 @@ class OracleBwdOps:
         out.copy_(acc)
 
 
-def _bwd_rank_main(rank, world, port, causal, out):
+def _bwd_rank_main(rank, world, port, causal, layout, out):
     import torch.distributed as dist
 
     import oracle
@@ -95,12 +95,10 @@ def _bwd_rank_main(rank, world, port, causal, out):
     try:
         q, k, v, do = _bwd_inputs(world)
         O, L = oracle.attention_fwd(q.numpy(), k.numpy(), v.numpy(), causal, 0.25)
-        n = q.shape[1] // world
-        sl = slice(rank * n, (rank + 1) * n)
-        c = lambda t: t[:, sl].contiguous()  # noqa: E731
+        c = lambda t, axis=1: _local(t, rank, world, layout, axis)  # noqa: E731
         dq, dk, dv = ring.ring_attention_bwd(c(q), c(k), c(v), c(torch.from_numpy(O)), c(do),
-                                             torch.from_numpy(L)[:, :, sl].contiguous(), causal=causal, scale=0.25,
-                                             ops=OracleBwdOps(0.25))
+                                             c(torch.from_numpy(L), 2), causal=causal, scale=0.25,
+                                             ops=OracleBwdOps(0.25), layout=layout)
         out[rank] = (dq.numpy(), dk.numpy(), dv.numpy())
     finally:
         dist.destroy_process_group()
@@ -108,85 +106,108 @@ def _bwd_rank_main(rank, world, port, causal, out):
 
 def _bwd_inputs(world):
     g = torch.Generator().manual_seed(12)
-    B, N, Hq, Hkv, d = 1, 40 * world, 4, 2, 8
+    B, N, Hq, Hkv, d = 1, 40 * world, 4, 2, 8  # 40 world rows: 2 world parts of 20
     return (torch.randn(B, N, Hq, d, generator=g, dtype=torch.float64),
             torch.randn(B, N, Hkv, d, generator=g, dtype=torch.float64),
             torch.randn(B, N, Hkv, d, generator=g, dtype=torch.float64),
             torch.randn(B, N, Hq, d, generator=g, dtype=torch.float64))
 
 
-@pytest.mark.parametrize("world,causal", [(1, True), (2, False), (2, True), (3, True)])
-def test_ring_backward_over_gloo_ranks_is_the_full_backward(world, causal):
+@pytest.mark.parametrize("world,causal,layout", [(1, True, "contiguous"), (2, False, "contiguous"),
+                                                 (2, True, "contiguous"), (3, True, "contiguous"),
+                                                 (2, True, "zigzag"), (3, True, "zigzag")])
+def test_ring_backward_over_gloo_ranks_is_the_full_backward(world, causal, layout):
     import torch.multiprocessing as mp
 
     import oracle
     port = _free_port()
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.spawn(_bwd_rank_main, args=(world, port, causal, out), nprocs=world, join=True)
+    mp.spawn(_bwd_rank_main, args=(world, port, causal, layout, out), nprocs=world, join=True)
     q, k, v, do = _bwd_inputs(world)
     DQ, DK, DV = oracle.attention_bwd(q.numpy(), k.numpy(), v.numpy(), do.numpy(), causal, 0.25)
-    n = q.shape[1] // world
     for r in range(world):
         dq, dk, dv = out[r]
-        sl = slice(r * n, (r + 1) * n)
-        np.testing.assert_allclose(dq, DQ[:, sl], rtol=0, atol=1e-6)
-        np.testing.assert_allclose(dk, DK[:, sl], rtol=0, atol=1e-6)
-        np.testing.assert_allclose(dv, DV[:, sl], rtol=0, atol=1e-6)
+        np.testing.assert_allclose(dq, _local(DQ, r, world, layout), rtol=0, atol=1e-6)
+        np.testing.assert_allclose(dk, _local(DK, r, world, layout), rtol=0, atol=1e-6)
+        np.testing.assert_allclose(dv, _local(DV, r, world, layout), rtol=0, atol=1e-6)
 
 
-def _rank_main(rank, world, port, causal, out):
+def _local(t, rank, world, layout, axis=1):
+    """This rank's parts of a whole-sequence tensor, concatenated in owned order."""
+    from exact_io_aware_80_b200 import ring
+    NP = ring.num_parts(world, layout)
+    n = t.shape[axis] // NP
+    idx = [slice(None)] * t.ndim
+    parts = []
+    for a in ring.owned_parts(rank, world, layout):
+        idx[axis] = slice(a * n, (a + 1) * n)
+        parts.append(t[tuple(idx)])
+    return np.concatenate(parts, axis=axis) if isinstance(t, np.ndarray) else torch.cat(parts, dim=axis).contiguous()
+
+
+def _fwd_inputs(world):
+    g = torch.Generator().manual_seed(11)
+    B, N, Hq, Hkv, d = 1, 48 * world, 4, 2, 16
+    return (torch.randn(B, N, Hq, d, generator=g, dtype=torch.float64),
+            torch.randn(B, N, Hkv, d, generator=g, dtype=torch.float64),
+            torch.randn(B, N, Hkv, d, generator=g, dtype=torch.float64))
+
+
+def _rank_main(rank, world, port, causal, layout, out):
     import torch.distributed as dist
 
     from exact_io_aware_80_b200 import ring
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
-        g = torch.Generator().manual_seed(11)
-        B, N, Hq, Hkv, d = 1, 48 * world, 4, 2, 16
-        q = torch.randn(B, N, Hq, d, generator=g, dtype=torch.float64)
-        k = torch.randn(B, N, Hkv, d, generator=g, dtype=torch.float64)
-        v = torch.randn(B, N, Hkv, d, generator=g, dtype=torch.float64)
-        n = N // world
-        sl = slice(rank * n, (rank + 1) * n)
-        o, lse = ring.ring_attention_fwd(q[:, sl].contiguous(), k[:, sl].contiguous(), v[:, sl].contiguous(),
-                                         causal=causal, scale=0.25, ops=OracleOps(0.25))
+        q, k, v = (_local(t, rank, world, layout) for t in _fwd_inputs(world))
+        o, lse = ring.ring_attention_fwd(q, k, v, causal=causal, scale=0.25, ops=OracleOps(0.25), layout=layout)
         out[rank] = (o.numpy(), lse.numpy())
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,causal", [(2, False), (2, True), (3, True)])
-def test_ring_over_gloo_ranks_is_exact_attention(world, causal):
+@pytest.mark.parametrize("world,causal,layout", [(2, False, "contiguous"), (2, True, "contiguous"),
+                                                 (3, True, "contiguous"), (2, True, "zigzag"), (3, True, "zigzag")])
+def test_ring_over_gloo_ranks_is_exact_attention(world, causal, layout):
     import torch.multiprocessing as mp
 
     import oracle
     port = _free_port()
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.spawn(_rank_main, args=(world, port, causal, out), nprocs=world, join=True)
-    g = torch.Generator().manual_seed(11)
-    B, N, Hq, Hkv, d = 1, 48 * world, 4, 2, 16
-    q = torch.randn(B, N, Hq, d, generator=g, dtype=torch.float64)
-    k = torch.randn(B, N, Hkv, d, generator=g, dtype=torch.float64)
-    v = torch.randn(B, N, Hkv, d, generator=g, dtype=torch.float64)
+    mp.spawn(_rank_main, args=(world, port, causal, layout, out), nprocs=world, join=True)
+    q, k, v = _fwd_inputs(world)
     O, L = oracle.attention_fwd(q.numpy(), k.numpy(), v.numpy(), causal, 0.25)
-    n = N // world
     for r in range(world):
         o, lse = out[r]
-        np.testing.assert_allclose(o, O[:, r * n:(r + 1) * n], rtol=0, atol=1e-5)
-        np.testing.assert_allclose(lse, L[:, :, r * n:(r + 1) * n], rtol=0, atol=1e-5)
+        np.testing.assert_allclose(o, _local(O, r, world, layout), rtol=0, atol=1e-5)
+        np.testing.assert_allclose(lse, _local(L, r, world, layout, axis=2), rtol=0, atol=1e-5)
 
 
-def test_schedule_visits_every_chunk_once():
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
+def test_schedule_covers_every_pair_once(layout):
     from exact_io_aware_80_b200 import ring
     for world in (1, 2, 3, 5):
         for causal in (False, True):
+            seen = {}
+            work = []
             for r in range(world):
-                sched = ring.ring_schedule(r, world, causal)
-                assert sorted(c for _, c, _ in sched) == list(range(world))
-                modes = {c: m for _, c, m in sched}
-                if causal:
-                    assert all(modes[c] == ("full" if c < r else "causal" if c == r else "skip") for c in modes)
-                else:
-                    assert set(modes.values()) == {"full"}
+                mine = ring.owned_parts(r, world, layout)
+                cnt = 0
+                for s, c, pairs in ring.ring_schedule(r, world, causal, layout):
+                    assert c == (r - s) % world
+                    theirs = ring.owned_parts(c, world, layout)
+                    for ia, ib, mode in pairs:
+                        a, b = mine[ia], theirs[ib]
+                        assert (a, b) not in seen
+                        seen[(a, b)] = mode
+                        assert mode == ("causal" if causal and a == b else "full")
+                        cnt += 1 if mode == "full" else 0.5
+                work.append(cnt)
+            NP = ring.num_parts(world, layout)
+            want = {(a, b) for a in range(NP) for b in range(NP) if not causal or b <= a}
+            assert set(seen) == want
+            if causal and layout == "zigzag":
+                assert max(work) == min(work)  # every rank gets the same causal work
