@@ -566,42 +566,72 @@ def run_ring_local(args, torch, w, q, k, v, dev, stream, world):
 
 
 def run_e2e(args, torch, fa, w, q, k, v, do, dev, stream, world, F):
-    """Same step through the public Python API with host buffers: pinned H2D of
-    q, k, v, dO, forward, backward, D2H of dQ, dK, dV, all inside the timed region."""
+    """Same step through the public Python API with host buffers: every step uploads q, k, v, dO from
+    pinned host memory, runs the forward and backward, and downloads dQ, dK, dV, all inside the timed
+    region.  Uploads, kernels and downloads run on three streams with two device buffer sets, so the
+    copies of neighbouring steps overlap the current step's kernels (events keep a buffer set from
+    being refilled before its kernels and download are done)."""
     hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
-    oq, ok_, ov = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (q, k, v))
-    dq_, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    qd, kd, vd, dod = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(do)
-    ws = torch.empty(fa.fa_bwd_workspace_bytes(w.B, w.Hq, w.Nq), device=dev, dtype=torch.uint8)
+    h_out = [tuple(torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (q, k, v)) for _ in range(2)]
+    bufs = []
+    for _ in range(2):
+        bufs.append({"q": torch.empty_like(q), "k": torch.empty_like(k), "v": torch.empty_like(v),
+                     "do": torch.empty_like(do), "dq": torch.empty_like(q), "dk": torch.empty_like(k),
+                     "dv": torch.empty_like(v),
+                     "ws": torch.empty(fa.fa_bwd_workspace_bytes(w.B, w.Hq, w.Nq), device=dev, dtype=torch.uint8)})
+    up, comp, down = (torch.cuda.Stream(device=dev) for _ in range(3))
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    downloaded = [torch.cuda.Event() for _ in range(2)]
+    seen = [False, False]
 
-    def step():
-        qd.copy_(hq, non_blocking=True)
-        kd.copy_(hk, non_blocking=True)
-        vd.copy_(hv, non_blocking=True)
-        dod.copy_(hdo, non_blocking=True)
-        o, lse = fa.attention_fwd(qd, kd, vd, causal=True)
-        fa.attention_bwd(qd, kd, vd, o, dod, lse, causal=True, workspace=ws, dq=dq_, dk=dk_, dv=dv_)
-        oq.copy_(dq_, non_blocking=True)
-        ok_.copy_(dk_, non_blocking=True)
-        ov.copy_(dv_, non_blocking=True)
+    def step(i):
+        b = i % 2
+        d = bufs[b]
+        with torch.cuda.stream(up):
+            if seen[b]:
+                up.wait_event(computed[b])  # the kernels of step i - 2 have read these inputs
+            d["q"].copy_(hq, non_blocking=True)
+            d["k"].copy_(hk, non_blocking=True)
+            d["v"].copy_(hv, non_blocking=True)
+            d["do"].copy_(hdo, non_blocking=True)
+            uploaded[b].record(up)
+        with torch.cuda.stream(comp):
+            comp.wait_event(uploaded[b])
+            if seen[b]:
+                comp.wait_event(downloaded[b])  # step i - 2's gradients have left these buffers
+            o, lse = fa.attention_fwd(d["q"], d["k"], d["v"], causal=True)
+            fa.attention_bwd(d["q"], d["k"], d["v"], o, d["do"], lse, causal=True, workspace=d["ws"], dq=d["dq"],
+                             dk=d["dk"], dv=d["dv"])
+            computed[b].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(computed[b])
+            for host, dev_t in zip(h_out[b], (d["dq"], d["dk"], d["dv"])):
+                host.copy_(dev_t, non_blocking=True)
+            downloaded[b].record(down)
+        seen[b] = True
 
-    for _ in range(args.warmup):
-        step()
+    for i in range(args.warmup):
+        step(i)
     torch.cuda.synchronize(dev)
     barrier(torch, world)
     K = args.steps
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(K):
-        step()
-    t1.record(stream)
+    up.wait_stream(down)  # the timed region starts after the warm-up's last download
+    t0.record(up)
+    for i in range(K):
+        step(args.warmup + i)
+    t1.record(down)  # after every step's download (and, through the events, every kernel)
     torch.cuda.synchronize(dev)
     barrier(torch, world)
     ms = max_over_ranks(torch, world, t0.elapsed_time(t1)) / K
+    if fa.device_status() != 0:
+        raise RuntimeError("kernel status word set during the end-to-end section")
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v, do))
-    d2h = sum(t.numel() * t.element_size() for t in (dq_, dk_, dv_))
+    d2h = sum(t.numel() * t.element_size() for t in (q, k, v))
     return {"value": round(world * 3.5 * F / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pipelining": "uploads, kernels and downloads on three streams, two device buffer sets"}
 
 
 def cpu_baseline(q, k, v, do, w):
