@@ -61,26 +61,23 @@ struct Params {
   Dropout drop;  // DROP only
 };
 
-// Store one 128-byte-aligned row segment of D 16-bit values from fp32 TMEM columns.
+// One row of D fp32 TMEM columns, times `mul`, as 16-bit values into a stage tile laid out as
+// a TMA box with 128-byte swizzle: 64-column panels of 128-byte rows, 16-byte chunk c of row r
+// at chunk c ^ (r & 7).
 template <typename T, int D>
-__device__ __forceinline__ void store_row(uint32_t taddr, uint16_t* dst, float mul, bool valid) {
+__device__ __forceinline__ void stage_row(uint32_t taddr, uint32_t stage, int r, float mul) {
 #pragma unroll
   for (int q = 0; q < D / 32; ++q) {
-    uint32_t r[32];
-    tmem_ld32(taddr + q * 32, r);
+    uint32_t x[32];
+    tmem_ld32(taddr + q * 32, x);
     tmem_wait_ld();
-    reg_fence(r);
-    if (valid) {
-      uint4* d4 = reinterpret_cast<uint4*>(dst + q * 32);
+    reg_fence(x);
+    auto pk = [&](int i) { return Elem<T>::pack(__uint_as_float(x[i]) * mul, __uint_as_float(x[i + 1]) * mul); };
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        uint4 w;
-        w.x = Elem<T>::pack(__uint_as_float(r[8 * v + 0]) * mul, __uint_as_float(r[8 * v + 1]) * mul);
-        w.y = Elem<T>::pack(__uint_as_float(r[8 * v + 2]) * mul, __uint_as_float(r[8 * v + 3]) * mul);
-        w.z = Elem<T>::pack(__uint_as_float(r[8 * v + 4]) * mul, __uint_as_float(r[8 * v + 5]) * mul);
-        w.w = Elem<T>::pack(__uint_as_float(r[8 * v + 6]) * mul, __uint_as_float(r[8 * v + 7]) * mul);
-        d4[v] = w;
-      }
+    for (int c4 = 0; c4 < 4; ++c4) {
+      const int cg = q * 4 + c4;  // 16-byte chunk of the row
+      st_shared_v4(stage + (cg >> 3) * kPanel + r * 128 + (((cg & 7) ^ (r & 7)) << 4), pk(8 * c4), pk(8 * c4 + 2),
+                   pk(8 * c4 + 4), pk(8 * c4 + 6));
     }
   }
 }
@@ -150,8 +147,9 @@ struct DkdvSmem {
   static constexpr int kOffLse = 6 * kTile;  // [2][128] fp32, log2 domain
   static constexpr int kOffD = kOffLse + 2 * kT * 4;
   static constexpr int kOffBar = kOffD + 2 * kT * 4;
+  // kBarOut: the elementwise threads have staged dK and dV (in the free Q / dO buffers)
   enum { kBarKV = 0, kBarQFull = 1, kBarQEmpty = 3, kBarS = 5, kBarDP = 6, kBarP = 7, kBarDS = 8, kBarDone = 9,
-         kBarDrain = 10, kBarLse = 11, kNumBars = 13 };
+         kBarDrain = 10, kBarLse = 11, kBarOut = 13, kNumBars = 14 };
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmem + 4;
   static constexpr int kBytes = kOffAbort + 4 + 1024;
@@ -163,6 +161,7 @@ template <typename T, int D, bool CAUSAL, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                          const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
                           Params p) {
   using L = DkdvSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -404,12 +403,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDone), 0, abort_flag, p.status));
     if (ok) {
+      // every MMA has run, so the Q and dO buffers are free: dV and dK leave through them by TMA
+      // (rows past Nk are clipped by the tensor maps)
       tc_fence_after();
-      const bool valid = key < p.Nk;
-      const long row = ((long)b * p.Nk + key) * p.Hkv + hk;
-      store_row<T, D>(tbase + lane_off + kColDV, static_cast<uint16_t*>(p.out1) + row * D,
-                      DROP ? p.drop.inv_keep : 1.f, valid);
-      store_row<T, D>(tbase + lane_off + kColDK, static_cast<uint16_t*>(p.out0) + row * D, p.scale, valid);
+      stage_row<T, D>(tbase + lane_off + kColDV, sb + L::kOffQ, jrow, DROP ? p.drop.inv_keep : 1.f);
+      stage_row<T, D>(tbase + lane_off + kColDK, sb + L::kOffDO, jrow, p.scale);
+      fence_proxy_async_smem();
+      mbar_arrive(bar(L::kBarOut));
+      if (tid == 0 && mbar_wait(bar(L::kBarOut), 0, abort_flag, p.status)) {
+#pragma unroll
+        for (int pn = 0; pn < D / 64; ++pn) {
+          tma_store_4d(&tmDV, sb + L::kOffQ + pn * kPanel, 64 * pn, hk, k0, b);
+          tma_store_4d(&tmDK, sb + L::kOffDO + pn * kPanel, 64 * pn, hk, k0, b);
+        }
+        bulk_commit();
+        bulk_wait_all();
+      }
     }
   }
 
@@ -433,8 +442,9 @@ struct DqSmem {
   static constexpr int kOffK = 2 * kTile;  // 3 stages
   static constexpr int kOffV = 5 * kTile;  // 2 stages
   static constexpr int kOffBar = 7 * kTile;
+  // kBarOut: the elementwise threads have staged dQ (in the free Q buffer)
   enum { kBarQ = 0, kBarKFull = 1, kBarKEmpty = 4, kBarVFull = 7, kBarVEmpty = 9, kBarS = 11, kBarDP = 13,
-         kBarDS = 14, kBarDone = 15, kBarDrain = 16, kNumBars = 17 };
+         kBarDS = 14, kBarDone = 15, kBarDrain = 16, kBarOut = 17, kNumBars = 18 };
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmem + 4;
   static constexpr int kBytes = kOffAbort + 4 + 1024;
@@ -447,7 +457,7 @@ template <typename T, int D, bool CAUSAL, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                        Params p) {
+                        const __grid_constant__ CUtensorMap tmDQ, Params p) {
   using L = DqSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -467,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n = (n_end + kT - 1) / kT;
 
   if (tid == 0) {
-    for (int i = 0; i < L::kNumBars; ++i) mbar_init(bar(i), i == L::kBarDS ? kT : 1);
+    for (int i = 0; i < L::kNumBars; ++i) mbar_init(bar(i), (i == L::kBarDS || i == L::kBarOut) ? kT : 1);
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -639,9 +649,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDone), 0, abort_flag, p.status));
     if (ok) {
+      // every MMA has run, so the Q buffer is free: dQ leaves through it by TMA (rows past Nq clipped)
       tc_fence_after();
-      const long orow = ((long)b * p.Nq + row) * p.Hq + h;
-      store_row<T, D>(tbase + lane_off + kColDQ, static_cast<uint16_t*>(p.out0) + orow * D, p.scale, row < p.Nq);
+      stage_row<T, D>(tbase + lane_off + kColDQ, sb + L::kOffQ, wq * 32 + lane, p.scale);
+      fence_proxy_async_smem();
+      mbar_arrive(bar(L::kBarOut));
+      if (tid == 0 && mbar_wait(bar(L::kBarOut), 0, abort_flag, p.status)) {
+#pragma unroll
+        for (int pn = 0; pn < D / 64; ++pn) tma_store_4d(&tmDQ, sb + L::kOffQ + pn * kPanel, 64 * pn, h, m0, b);
+        bulk_commit();
+        bulk_wait_all();
+      }
     }
   }
 
@@ -658,14 +676,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 // host side
 // ---------------------------------------------------------------------------
 struct Maps {
-  CUtensorMap q, k, v, dO;
+  CUtensorMap q, k, v, dO, dq, dk, dv;
 };
 
-bool make_maps(Maps& m, const BwdArgs& a) {
+// Loads of Q, K, V, dO; stores of whichever of dQ, dK, dV the launch writes.
+bool make_maps(Maps& m, const BwdArgs& a, bool kv_out, bool q_out) {
   const bool bf16 = a.bf16 != 0;
-  return make_map(&m.q, a.q, bf16, a.d, a.Hq, a.Nq, a.B, kT) && make_map(&m.k, a.k, bf16, a.d, a.Hkv, a.Nk, a.B, kT) &&
-         make_map(&m.v, a.v, bf16, a.d, a.Hkv, a.Nk, a.B, kT) &&
-         make_map(&m.dO, a.dout, bf16, a.d, a.Hq, a.Nq, a.B, kT);
+  bool ok = make_map(&m.q, a.q, bf16, a.d, a.Hq, a.Nq, a.B, kT) && make_map(&m.k, a.k, bf16, a.d, a.Hkv, a.Nk, a.B, kT) &&
+            make_map(&m.v, a.v, bf16, a.d, a.Hkv, a.Nk, a.B, kT) &&
+            make_map(&m.dO, a.dout, bf16, a.d, a.Hq, a.Nq, a.B, kT);
+  if (ok && kv_out)
+    ok = make_map(&m.dk, a.dk, bf16, a.d, a.Hkv, a.Nk, a.B, kT) && make_map(&m.dv, a.dv, bf16, a.d, a.Hkv, a.Nk, a.B, kT);
+  if (ok && q_out) ok = make_map(&m.dq, a.dq, bf16, a.d, a.Hq, a.Nq, a.B, kT);
+  return ok;
 }
 
 Params params(const BwdArgs& a, void* out0, void* out1) {
@@ -676,26 +699,26 @@ Params params(const BwdArgs& a, void* out0, void* out1) {
 template <typename T, int D, bool CAUSAL>
 cudaError_t launch_dkdv(const BwdArgs& a, cudaStream_t s) {
   Maps m;
-  if (!make_maps(m, a)) return cudaErrorInvalidValue;
+  if (!make_maps(m, a, true, false)) return cudaErrorInvalidValue;
   auto kern = a.drop_p > 0.f ? bwd_dkdv_sm100_kernel<T, D, CAUSAL, true> : bwd_dkdv_sm100_kernel<T, D, CAUSAL, false>;
   const int smem = DkdvSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.Hkv, (a.Nk + kT - 1) / kT, a.B);
-  kern<<<grid, kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, params(a, a.dk, a.dv));
+  kern<<<grid, kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, m.dk, m.dv, params(a, a.dk, a.dv));
   return cudaGetLastError();
 }
 
 template <typename T, int D, bool CAUSAL>
 cudaError_t launch_dq(const BwdArgs& a, cudaStream_t s) {
   Maps m;
-  if (!make_maps(m, a)) return cudaErrorInvalidValue;
+  if (!make_maps(m, a, false, true)) return cudaErrorInvalidValue;
   auto kern = a.drop_p > 0.f ? bwd_dq_sm100_kernel<T, D, CAUSAL, true> : bwd_dq_sm100_kernel<T, D, CAUSAL, false>;
   const int smem = DqSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.Hq, (a.Nq + kT - 1) / kT, a.B);
-  kern<<<grid, kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, params(a, a.dq, nullptr));
+  kern<<<grid, kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, m.dq, params(a, a.dq, nullptr));
   return cudaGetLastError();
 }
 
