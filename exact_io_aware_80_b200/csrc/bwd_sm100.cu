@@ -327,6 +327,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < nt; ++t) {
       const int buf = t & 1;
       const int i0 = (mstart + t % per_head) * kT;
+      uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit cc = (query i0 + cc, this key) kept
+      if constexpr (DROP) {
+        // drawn before the scores arrive, four independent Philox calls at a time.  Lanes 4m ..
+        // 4m + 3 hold the four keys of one key quad, which share every call: each lane makes the
+        // calls of every fourth query pair, which give two bits (the pair's queries) for each key
+        // of the quad, and the lanes swap them (lane ^ 1, ^ 2, ^ 3)
+        const uint32_t bh = (uint32_t)(b * p.Hq + hk * G + t / per_head), jq = (uint32_t)key >> 2;
+        const int r = key & 3;  // == lane & 3
+        const uint32_t thr = p.drop.thr;
+        uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u};  // bits of keys 4 jq + k at this
+        uint32_t a2[4] = {0u, 0u, 0u, 0u}, a3[4] = {0u, 0u, 0u, 0u};  // lane's query pairs, by word
+#pragma unroll 1
+        for (int t2 = 0; t2 < 4; ++t2) {
+#pragma unroll
+          for (int wd = 0; wd < 4; ++wd) {
+            // the call of the 2 x 4 block (queries i0 + cc, + 1) x (keys 4 jq .. 4 jq + 3)
+            const int cc = 32 * wd + 8 * t2 + 2 * r;
+            const uint4 w = philox4x32_10(jq, (uint32_t)(i0 + cc) >> 1, bh, p.drop.offset, p.drop.seed_lo,
+                                          p.drop.seed_hi);
+            const int sh = cc & 31;
+            a0[wd] |= keep_pair(w.x & 0xFFFFu, w.z & 0xFFFFu, thr) << sh;
+            a1[wd] |= keep_pair(w.x >> 16, w.z >> 16, thr) << sh;
+            a2[wd] |= keep_pair(w.y & 0xFFFFu, w.w & 0xFFFFu, thr) << sh;
+            a3[wd] |= keep_pair(w.y >> 16, w.w >> 16, thr) << sh;
+          }
+        }
+#pragma unroll
+        for (int wd = 0; wd < 4; ++wd) {
+          auto pick = [&](int k) { return k == 0 ? a0[wd] : k == 1 ? a1[wd] : k == 2 ? a2[wd] : a3[wd]; };
+          uint32_t kw = pick(r);
+          kw |= __shfl_xor_sync(0xffffffffu, pick(r ^ 1), 1);
+          kw |= __shfl_xor_sync(0xffffffffu, pick(r ^ 2), 2);
+          kw |= __shfl_xor_sync(0xffffffffu, pick(r ^ 3), 3);
+          keep[wd] = kw;
+        }
+      }
       float nl = 0.f, nd = 0.f;
       if (t + 1 < nt) fetch(t + 1, nl, nd);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarLse + buf), (t >> 1) & 1, abort_flag, p.status));
@@ -349,29 +385,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < kT; ++cc)
           if (cc < lim) pv[cc] = 0.f;
-      }
-      uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit cc = (query i0 + cc, this key) kept
-      if constexpr (DROP) {
-        // lanes 2m and 2m + 1 hold the two keys of one key pair, which share every Philox call:
-        // each lane makes every other call (query pairs) and hands the other key's bits to lane ^ 1
-        const uint32_t bh = (uint32_t)(b * p.Hq + hk * G + t / per_head), jp = (uint32_t)key >> 1;
-        const int e = key & 1;  // == lane & 1
-#pragma unroll
-        for (int wd = 0; wd < 4; ++wd) {
-          uint32_t own = 0, other = 0;
-#pragma unroll 1
-          for (int t2 = 0; t2 < 8; ++t2) {
-            // the call of the 2 x 2 block (queries i0 + cc, + 1) x (keys 2 jp, 2 jp + 1)
-            const int cc = 32 * wd + 4 * t2 + 2 * e;
-            const uint4 w = philox4x32_10(jp, (uint32_t)(i0 + cc) >> 1, bh, p.drop.offset, p.drop.seed_lo,
-                                          p.drop.seed_hi);
-            const uint32_t even = (uint32_t)(w.x >= p.drop.thr) | ((uint32_t)(w.z >= p.drop.thr) << 1);
-            const uint32_t odd = (uint32_t)(w.y >= p.drop.thr) | ((uint32_t)(w.w >= p.drop.thr) << 1);
-            own |= (e ? odd : even) << (cc & 31);
-            other |= (e ? even : odd) << (cc & 31);
-          }
-          keep[wd] = own | __shfl_xor_sync(0xffffffffu, other, 1);
-        }
       }
       {
         auto pd = [&](int c) { return DROP && !((keep[c >> 5] >> (c & 31)) & 1u) ? 0.f : pv[c]; };
@@ -597,6 +610,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const uint32_t tS = tbase + lane_off + col_s(j & 1);
+      const int kb = j * kT;
+      uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit cc = (this query, key kb + cc) kept
+      if constexpr (DROP) {
+        // drawn before the scores arrive, four independent Philox calls at a time.  Lanes 2m and
+        // 2m + 1 hold one query pair: each makes the calls of every other key quad and hands the
+        // other row's bits to lane ^ 1
+        const uint32_t bh = (uint32_t)(b * p.Hq + h), rh = (uint32_t)row >> 1;
+        const int e = row & 1;  // == lane & 1
+        uint32_t own[4] = {0u, 0u, 0u, 0u}, other[4] = {0u, 0u, 0u, 0u};
+#pragma unroll 1
+        for (int t2 = 0; t2 < 4; ++t2) {
+#pragma unroll
+          for (int wd = 0; wd < 4; ++wd) {
+            const int cc = 32 * wd + 8 * t2 + 4 * e;  // keys kb + cc .. cc + 3
+            const uint4 w = philox4x32_10((uint32_t)(kb + cc) >> 2, rh, bh, p.drop.offset, p.drop.seed_lo,
+                                          p.drop.seed_hi);
+            const uint32_t even = keep_quad(w.x, w.y, p.drop.thr), odd = keep_quad(w.z, w.w, p.drop.thr);
+            own[wd] |= (e ? odd : even) << (cc & 31);
+            other[wd] |= (e ? even : odd) << (cc & 31);
+          }
+        }
+#pragma unroll
+        for (int wd = 0; wd < 4; ++wd) keep[wd] = own[wd] | __shfl_xor_sync(0xffffffffu, other[wd], 1);
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + (j & 1)), (j >> 1) & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
@@ -609,7 +646,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         pv[cc] = x.x;
         pv[cc + 1] = x.y;
       }
-      const int kb = j * kT;
       if (kb + kT > p.Nk || (CAUSAL && kb + kT - 1 > m0 + off)) {
         int lim = p.Nk - kb;
         if (CAUSAL) lim = min(lim, row + off + 1 - kb);
@@ -620,28 +656,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), j & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
-      uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit cc = (this query, key kb + cc) kept
-      if constexpr (DROP) {
-        // lanes 2m and 2m + 1 hold one query pair: each makes every other call (key pairs) and
-        // hands the other row's bits to lane ^ 1
-        const uint32_t bh = (uint32_t)(b * p.Hq + h), rh = (uint32_t)row >> 1;
-        const int e = row & 1;  // == lane & 1
-#pragma unroll
-        for (int wd = 0; wd < 4; ++wd) {
-          uint32_t own = 0, other = 0;
-#pragma unroll 1
-          for (int t2 = 0; t2 < 8; ++t2) {
-            const int cc = 32 * wd + 4 * t2 + 2 * e;
-            const uint4 w = philox4x32_10((uint32_t)(kb + cc) >> 1, rh, bh, p.drop.offset, p.drop.seed_lo,
-                                          p.drop.seed_hi);
-            const uint32_t even = (uint32_t)(w.x >= p.drop.thr) | ((uint32_t)(w.y >= p.drop.thr) << 1);
-            const uint32_t odd = (uint32_t)(w.z >= p.drop.thr) | ((uint32_t)(w.w >= p.drop.thr) << 1);
-            own |= (e ? odd : even) << (cc & 31);
-            other |= (e ? even : odd) << (cc & 31);
-          }
-          keep[wd] = own | __shfl_xor_sync(0xffffffffu, other, 1);
-        }
-      }
       write_ds<T, false, DROP>(tbase + lane_off + kColDP, tS, pv, nullptr, ndrow, keep, p.drop.inv_keep);
       tmem_wait_st();
       tc_fence_before();

@@ -46,14 +46,28 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_
   return make_uint4(c0, c1, c2, c3);
 }
 
-// Dropout of one (b, h_q): one Philox call per 2 x 2 block of (query i, key j),
-// counter (j >> 1, i >> 1, b * Hq + h, offset), key = the 64-bit seed; word
-// 2 (i & 1) + (j & 1) decides (i, j): kept iff it is >= thr = floor(p 2^32).
+// Dropout of one (b, h_q): one Philox call per 2 x 4 block of (query i, key j),
+// counter (j >> 2, i >> 1, b * Hq + h, offset), key = the 64-bit seed.  The
+// call's four words are eight 16-bit values (low half first); value
+// e = 4 (i & 1) + (j & 3), the half e & 1 of word e >> 1, decides (i, j): kept
+// iff it is >= thr = floor(p 2^16).
 struct Dropout {
-  uint32_t thr;       // floor(p * 2^32)
+  uint32_t thr;       // floor(p * 2^16)
   float inv_keep;     // 1 / (1 - p)
   uint32_t seed_lo, seed_hi, offset;
 };
+
+// Keep bits of one row of a 2 x 4 block from the row's two words (a: keys 0-1, b: keys 2-3):
+// bit k = key k of the quad.
+__device__ __forceinline__ uint32_t keep_quad(uint32_t a, uint32_t b, uint32_t thr) {
+  return (uint32_t)((a & 0xFFFFu) >= thr) | ((uint32_t)((a >> 16) >= thr) << 1) |
+         ((uint32_t)((b & 0xFFFFu) >= thr) << 2) | ((uint32_t)((b >> 16) >= thr) << 3);
+}
+// Keep bits of one key of a 2 x 4 block for both rows, from the key's value in the even-row word
+// (ve) and the odd-row word (vo): bit 0 = even row, bit 1 = odd row.
+__device__ __forceinline__ uint32_t keep_pair(uint32_t ve, uint32_t vo, uint32_t thr) {
+  return (uint32_t)(ve >= thr) | ((uint32_t)(vo >= thr) << 1);
+}
 
 // ---------------------------------------------------------------------------
 // element types

@@ -51,7 +51,7 @@ fa_status check_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
 
 fa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
 
-// Dropout parameters: keep iff the Philox word >= floor(p 2^32), weights scaled by 1 / (1 - p).
+// Dropout parameters: keep iff the 16-bit Philox value >= floor(p 2^16), weights scaled by 1 / (1 - p).
 struct DropParams {
   float p = 0.f;
   uint32_t thr = 0;
@@ -60,9 +60,9 @@ struct DropParams {
 };
 bool make_drop(float p, unsigned long long seed, uint32_t offset, DropParams* out) {
   if (!(p >= 0.f && p < 1.f)) return false;
-  const double t = std::floor((double)p * 4294967296.0);
+  const double t = std::floor((double)p * 65536.0);  // 16-bit keep threshold
   out->p = p;
-  out->thr = (uint32_t)(t > 4294967295.0 ? 4294967295.0 : t);
+  out->thr = (uint32_t)(t > 65535.0 ? 65535.0 : t);
   out->inv_keep = (float)(1.0 / (1.0 - (double)p));
   out->seed_lo = (uint32_t)(seed & 0xFFFFFFFFull);
   out->seed_hi = (uint32_t)(seed >> 32);

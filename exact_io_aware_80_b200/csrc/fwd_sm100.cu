@@ -46,9 +46,9 @@
 // not mark, and a work tile with none writes O = 0 and LSE = -inf directly.
 //
 // Instantiated with DROP, it applies dropout to P ("FlashAttention 심층 분석",
-// section 2: dropout is one of the fused steps): every 4-key step of the
-// exponentials draws two Philox4x32-10 words per row (common.cuh: one call per
-// 2 x 2 block of query/key pairs) and zeroes the dropped entries of P before
+// section 2: dropout is one of the fused steps): Philox4x32-10 calls (common.cuh:
+// one call per 2 x 4 block of query/key pairs, one 16-bit value per pair) give
+// every row its 128 keep bits per key tile, and the dropped entries of P are zeroed before
 // the P V product; l keeps the sum of the undropped p, so LSE is that of the
 // scores, and the epilogue multiplies O by 1 / (1 - p).
 #include <cuda.h>
@@ -433,6 +433,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (F8) cq = c * p.q_scale[((long)b * p.Hq + h) * p.nqb + min(row_first / kBM, p.nqb - 1)];
       float m_ref = -INFINITY, l = 0.f;
       for (int j = j0; j < nblk; j = next_vis(x, j + 1, nblk), ++g) {
+        uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit c = (this row, key j kBN + c) kept
+        if constexpr (DROP) {
+          // drawn before the scores arrive (they need neither), four independent Philox calls at a
+          // time.  Lanes 2m and 2m + 1 hold the two rows of one query pair, which share every call
+          // (a key quad): each lane makes the calls of every other quad, keeps both rows' bits and
+          // hands the other row's to its partner (lane ^ 1)
+          const uint32_t rh = (uint32_t)row >> 1, bh = (uint32_t)(b * p.Hq + h);
+          const int e = row & 1;  // == lane & 1
+          uint32_t own[4] = {0u, 0u, 0u, 0u}, other[4] = {0u, 0u, 0u, 0u};
+#pragma unroll 1
+          for (int t2 = 0; t2 < 4; ++t2) {
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) {
+              const int c = 32 * wd + 8 * t2 + 4 * e;  // keys j kBN + c .. c + 3: this lane's quad
+              const uint4 w = philox4x32_10((uint32_t)(j * kBN + c) >> 2, rh, bh, p.drop.offset, p.drop.seed_lo,
+                                            p.drop.seed_hi);
+              const uint32_t even = keep_quad(w.x, w.y, p.drop.thr), odd = keep_quad(w.z, w.w, p.drop.thr);
+              own[wd] |= (e ? odd : even) << (c & 31);
+              other[wd] |= (e ? even : odd) << (c & 31);
+            }
+          }
+#pragma unroll
+          for (int wd = 0; wd < 4; ++wd) keep[wd] = own[wd] | __shfl_xor_sync(0xffffffffu, other[wd], 1);
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + t), g & 1, abort_flag, p.status));
         if (!ok) break;
         tc_fence_after();
@@ -482,29 +506,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (resc) m_ref = mxs;
         l *= corr;
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-        uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit c = (this row, key kbase + c) kept
-        if constexpr (DROP) {
-          // lanes 2m and 2m + 1 hold the two rows of one query pair, which share every Philox call:
-          // each lane makes every other call, keeps both rows' bits and hands the other row's to
-          // its partner (lane ^ 1)
-          const uint32_t rh = (uint32_t)row >> 1, bh = (uint32_t)(b * p.Hq + h);
-          const int e = row & 1;  // == lane & 1
-#pragma unroll
-          for (int wd = 0; wd < 4; ++wd) {
-            uint32_t own = 0, other = 0;
-#pragma unroll 1
-            for (int t2 = 0; t2 < 8; ++t2) {
-              const int c = 32 * wd + 4 * t2 + 2 * e;  // keys kbase + c, + 1: this lane's key pair
-              const uint4 w = philox4x32_10((uint32_t)(kbase + c) >> 1, rh, bh, p.drop.offset, p.drop.seed_lo,
-                                            p.drop.seed_hi);
-              const uint32_t even = (uint32_t)(w.x >= p.drop.thr) | ((uint32_t)(w.y >= p.drop.thr) << 1);
-              const uint32_t odd = (uint32_t)(w.z >= p.drop.thr) | ((uint32_t)(w.w >= p.drop.thr) << 1);
-              own |= (e ? odd : even) << (c & 31);
-              other |= (e ? even : odd) << (c & 31);
-            }
-            keep[wd] = own | __shfl_xor_sync(0xffffffffu, other, 1);
-          }
-        }
         const float2 c2 = make_float2(cj, cj), nm2 = make_float2(-mu, -mu);
         float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
 #pragma unroll

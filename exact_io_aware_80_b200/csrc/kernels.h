@@ -20,7 +20,7 @@ struct AttnArgs {
   int bf16;  // 1: bf16, 0: fp16
   int* status;
   const uint8_t* block_mask = nullptr;  // block-sparse forward: [B, Hq, ceil(Nq/128), ceil(Nk/128)]
-  // dropout (drop_p > 0): keep threshold floor(p 2^32), 1 / (1 - p), Philox key and counter offset
+  // dropout (drop_p > 0): keep threshold floor(p 2^16), 1 / (1 - p), Philox key and counter offset
   float drop_p = 0.f;
   uint32_t drop_thr = 0;
   float drop_inv_keep = 1.f;

@@ -188,11 +188,12 @@ fa_status fa_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
 /*
  * Dropout ("FlashAttention 심층 분석", section 2: dropout is one of the fused steps;
  * section 4: the backward pass regenerates what it needs).  The mask comes from
- * Philox4x32-10 (Salmon et al., SC 2011): one call per 2 x 2 block of (query i,
- * key j) of head (b, h), counter (j >> 1, i >> 1, b * Hq + h, offset), key =
- * (seed & 0xffffffff, seed >> 32); element (i, j) takes word 2 (i & 1) + (j & 1)
- * and is kept iff that word >= floor(p_drop * 2^32) (p_drop as passed, in
- * [0, 1); FA_ERR_INVALID otherwise).  The forward computes
+ * Philox4x32-10 (Salmon et al., SC 2011): one call per 2 x 4 block of (query i,
+ * key j) of head (b, h), counter (j >> 2, i >> 1, b * Hq + h, offset), key =
+ * (seed & 0xffffffff, seed >> 32); the call's four words are read as eight
+ * 16-bit values (low half of a word first), element (i, j) takes value
+ * 4 (i & 1) + (j & 3) and is kept iff that value >= floor(p_drop * 2^16)
+ * (p_drop as passed, in [0, 1); FA_ERR_INVALID otherwise).  The forward computes
  * O = (P * M / (1 - p_drop)) V and the LSE of the undropped scores; the
  * backward (same seed, offset and p_drop) regenerates M and returns the
  * gradients of sum(dO * O) for that forward.  p_drop = 0 gives fa_fwd /

@@ -14,10 +14,11 @@ name no generator and no keep rule.  Readings (listed in the design doc):
   definition: per round, (c0, c1, c2, c3) -> (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2),
   hi(M0 c0) ^ c3 ^ k1, lo(M0 c0)) with M0 = 0xD2511F53, M1 = 0xCD9E8D57, and
   the key bumped by (0x9E3779B9, 0xBB67AE85) before every round but the first;
-* one call covers a 2 x 2 block of (query i, key j) for one (b, h_q):
-  counter = (j >> 1, i >> 1, b * Hq + h, offset), key = (seed_lo, seed_hi);
-  output word 2 (i & 1) + (j & 1) belongs to (i, j);
-* keep (i, j) iff that word >= floor(p * 2^32) (p in [0, 1)); kept weights are
+* one call covers a 2 x 4 block of (query i, key j) for one (b, h_q):
+  counter = (j >> 2, i >> 1, b * Hq + h, offset), key = (seed_lo, seed_hi);
+  its four 32-bit words are read as eight 16-bit values, the low half of a
+  word first, and value e = 4 (i & 1) + (j & 3) belongs to (i, j);
+* keep (i, j) iff that value >= floor(p * 2^16) (p in [0, 1)); kept weights are
   scaled by 1 / (1 - p), dropped ones are 0;
 * O = (P * M / (1 - p)) V with P the softmax of the scores (unchanged by
   dropout) and LSE that of the scores; backward by the chain rule with the
@@ -54,10 +55,10 @@ def philox4x32(c0, c1, c2, c3, k0: int, k1: int, rounds: int = 10):
 
 
 def keep_threshold(p: float) -> int:
-    """floor(p * 2^32), capped to 2^32 - 1."""
+    """floor(p * 2^16), capped to 2^16 - 1."""
     if not 0.0 <= p < 1.0:
         raise ValueError("dropout probability must be in [0, 1)")
-    return min(int(np.floor(p * 4294967296.0)), 0xFFFFFFFF)
+    return min(int(np.floor(p * 65536.0)), 0xFFFF)
 
 
 def keep_mask(b: int, h: int, Hq: int, Nq: int, Nk: int, p: float, seed: int, offset: int) -> np.ndarray:
@@ -65,11 +66,12 @@ def keep_mask(b: int, h: int, Hq: int, Nq: int, Nk: int, p: float, seed: int, of
     i = np.arange(Nq, dtype=np.uint64)[:, None]
     j = np.arange(Nk, dtype=np.uint64)[None, :]
     ii, jj = np.broadcast_arrays(i, j)
-    words = philox4x32(jj >> np.uint64(1), ii >> np.uint64(1), np.full(ii.shape, b * Hq + h, np.uint64),
+    words = philox4x32(jj >> np.uint64(2), ii >> np.uint64(1), np.full(ii.shape, b * Hq + h, np.uint64),
                        np.full(ii.shape, offset, np.uint64), seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
-    sel = (2 * (ii & np.uint64(1)) + (jj & np.uint64(1))).astype(np.int64)
-    w = np.choose(sel, words)
-    return w >= np.uint64(keep_threshold(p))
+    e = (4 * (ii & np.uint64(1)) + (jj & np.uint64(3))).astype(np.int64)
+    w = np.choose(e >> 1, words)
+    value = (w >> (np.uint64(16) * (e & 1).astype(np.uint64))) & np.uint64(0xFFFF)
+    return value >= np.uint64(keep_threshold(p))
 
 
 def attention_fwd_dropout(q, k, v, causal: bool, scale: float, p: float, seed: int, offset: int):

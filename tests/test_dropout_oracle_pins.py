@@ -44,15 +44,34 @@ def test_keep_rate_is_binomial():
     assert (M != dr.keep_mask(0, 3, 8, Nq, Nk, p, 0x1234_5678_9ABC, 8)).mean() > 0.3
 
 
-def test_mask_word_selection():
-    # (i, j) takes word 2 (i & 1) + (j & 1) of the call at counter (j >> 1, i >> 1, bh, offset)
+def test_mask_value_selection():
+    # (i, j) takes 16-bit value e = 4 (i & 1) + (j & 3) of the call at counter (j >> 2, i >> 1, bh,
+    # offset): the low half of word e >> 1 for even e, the high half for odd e.  Counter (3, 10)
+    # covers queries 20, 21 and keys 12 .. 15.
     seed, off, bh = 0xDEADBEEF00C0FFEE, 5, 2 * 4 + 1
     w = dr.philox4x32(np.array([3]), np.array([10]), np.array([bh]), np.array([off]), seed & 0xFFFFFFFF, seed >> 32)
-    thr = dr.keep_threshold(0.5)
-    M = dr.keep_mask(2, 1, 4, 22, 8, 0.5, seed, off)
-    for di in (0, 1):
-        for dj in (0, 1):
-            assert M[20 + di, 6 + dj] == (int(w[2 * di + dj][0]) >= thr)
+    words = [int(x[0]) for x in w]
+    values = [words[0] & 0xFFFF, words[0] >> 16, words[1] & 0xFFFF, words[1] >> 16,
+              words[2] & 0xFFFF, words[2] >> 16, words[3] & 0xFFFF, words[3] >> 16]
+    for pr in (0.25, 0.5, 0.9):
+        thr = dr.keep_threshold(pr)
+        M = dr.keep_mask(2, 1, 4, 22, 16, pr, seed, off)
+        for di in (0, 1):
+            for dj in range(4):
+                assert M[20 + di, 12 + dj] == (values[4 * di + dj] >= thr)
+    # the neighbouring blocks come from other counters
+    M = dr.keep_mask(2, 1, 4, 24, 20, 0.5, seed, off)
+    w2 = dr.philox4x32(np.array([4]), np.array([11]), np.array([bh]), np.array([off]), seed & 0xFFFFFFFF, seed >> 32)
+    assert M[23, 19] == ((int(w2[3][0]) >> 16) >= dr.keep_threshold(0.5))
+
+
+def test_keep_threshold():
+    assert dr.keep_threshold(0.0) == 0
+    assert dr.keep_threshold(0.1) == 6553
+    assert dr.keep_threshold(0.5) == 32768
+    assert dr.keep_threshold(1 - 2 ** -20) == 65535
+    with pytest.raises(ValueError):
+        dr.keep_threshold(1.0)
 
 
 def test_p_zero_is_plain_attention():
