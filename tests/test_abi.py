@@ -75,6 +75,11 @@ FAKE = 0x10000  # never dereferenced: validation fails first
     (dict(d=256), -2),
     (dict(dt=7), -2),
     (dict(B=0), -1),
+    (dict(Nq=0), -1),
+    (dict(Nk=0), -1),
+    (dict(Hkv=0), -1),
+    (dict(Nq=(1 << 30) + 1, Nk=(1 << 30) + 1), -2),
+    (dict(B=65536), -2),
     (dict(q=FAKE + 8), -3),
 ])
 def test_fwd_rejects_bad_arguments(lib, kw, code):
