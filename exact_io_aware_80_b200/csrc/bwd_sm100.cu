@@ -45,6 +45,12 @@ using namespace sm100;
 
 constexpr int kT = 128;        // rows of every tile (keys or queries) = TMEM lanes
 constexpr int kThreads = 192;  // warps 0-3 elementwise, 4 TMA, 5 MMA
+// dK/dV with dropout: a third warpgroup (warps 8-11, one warp per SM sub-partition) draws the
+// keep bits; warps 6-7 idle.  The 384 threads launch with 168 registers each; each role's branch
+// then moves its warpgroup to its own budget.
+constexpr int kThreadsDrop = 384;
+constexpr int kRegsElem = 256, kRegsCtrl = 104, kRegsRng = 104;
+static_assert(128 * (kRegsElem + kRegsCtrl + kRegsRng) <= kThreadsDrop * 168, "register split exceeds the launch");
 constexpr int kWarpLoad = 4;
 constexpr int kWarpMma = 5;
 constexpr int kPanel = 128 * 128;  // [128 rows][64 cols] 16-bit panel, bytes
@@ -146,10 +152,12 @@ struct DkdvSmem {
   static constexpr int kOffDO = 4 * kTile;  // 2 stages
   static constexpr int kOffLse = 6 * kTile;  // [2][128] fp32, log2 domain
   static constexpr int kOffD = kOffLse + 2 * kT * 4;
-  static constexpr int kOffBar = kOffD + 2 * kT * 4;
-  // kBarOut: the elementwise threads have staged dK and dV (in the free Q / dO buffers)
+  static constexpr int kOffKeep = kOffD + 2 * kT * 4;  // dropout: [2][128 keys] x 128 keep bits
+  static constexpr int kOffBar = kOffKeep + 2 * kT * 16;
+  // kBarOut: the elementwise threads have staged dK and dV (in the free Q / dO buffers);
+  // kBarKeepFull / kBarKeepEmpty: a slot of the keep-bit ring written / read
   enum { kBarKV = 0, kBarQFull = 1, kBarQEmpty = 3, kBarS = 5, kBarDP = 6, kBarP = 7, kBarDS = 8, kBarDone = 9,
-         kBarDrain = 10, kBarLse = 11, kBarOut = 13, kNumBars = 14 };
+         kBarDrain = 10, kBarLse = 11, kBarOut = 13, kBarKeepFull = 14, kBarKeepEmpty = 16, kNumBars = 18 };
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmem + 4;
   static constexpr int kBytes = kOffAbort + 4 + 1024;
@@ -158,7 +166,7 @@ struct DkdvSmem {
 constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256, kColDK = 384;
 
 template <typename T, int D, bool CAUSAL, bool DROP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                           const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
@@ -208,7 +216,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(gb + L::kOffTmem);
 
-  if (warp == kWarpLoad) {
+  if (warp >= 4 && warp < 8) {
+   if constexpr (DROP) regs_decrease<kRegsCtrl>();
+   if (warp == kWarpLoad) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int last_u[2] = {-1, -1};
@@ -298,7 +308,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar(L::kBarDrain));
       wait_drain(bar(L::kBarDrain), 0, p.status);
     }
+  }
+  } else if (DROP && warp >= 8) {
+    if constexpr (DROP) regs_decrease<kRegsRng>();
+    // ------------------------------------------------------------------ keep bits (dropout)
+    // thread rt draws the keep bits of key k0 + rt for every query tile into ring slot t & 1.
+    // Lanes 4m .. 4m + 3 hold the four keys of one key quad, which share every Philox call:
+    // each lane makes the calls of every fourth query pair, which give two bits (the pair's
+    // queries) for each key of the quad, and the lanes swap them (lane ^ 1, ^ 2, ^ 3); four
+    // independent calls are in flight at a time.
+    const int rt = tid - 256;
+    const int key = k0 + rt;
+    const uint32_t jq = (uint32_t)key >> 2, thr = p.drop.thr;
+    const int r = key & 3;  // == lane & 3
+    uint4* ring = reinterpret_cast<uint4*>(gb + L::kOffKeep);
+    for (int t = 0; t < nt; ++t) {
+      const int slot = t & 1;
+      if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar(L::kBarKeepEmpty + slot), ((t >> 1) - 1) & 1,
+                                                       abort_flag, p.status)))
+        break;
+      const int i0 = (mstart + t % per_head) * kT;
+      const uint32_t bh = (uint32_t)(b * p.Hq + hk * G + t / per_head);
+      uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u};  // bits of keys 4 jq + k at this
+      uint32_t a2[4] = {0u, 0u, 0u, 0u}, a3[4] = {0u, 0u, 0u, 0u};  // lane's query pairs, by word
+#pragma unroll 1
+      for (int t2 = 0; t2 < 4; ++t2) {
+#pragma unroll
+        for (int wd = 0; wd < 4; ++wd) {
+          // the call of the 2 x 4 block (queries i0 + cc, + 1) x (keys 4 jq .. 4 jq + 3)
+          const int cc = 32 * wd + 8 * t2 + 2 * r;
+          const uint4 w = philox4x32_10(jq, (uint32_t)(i0 + cc) >> 1, bh, p.drop.offset, p.drop.seed_lo,
+                                        p.drop.seed_hi);
+          const int sh = cc & 31;
+          a0[wd] |= keep_pair(w.x & 0xFFFFu, w.z & 0xFFFFu, thr) << sh;
+          a1[wd] |= keep_pair(w.x >> 16, w.z >> 16, thr) << sh;
+          a2[wd] |= keep_pair(w.y & 0xFFFFu, w.w & 0xFFFFu, thr) << sh;
+          a3[wd] |= keep_pair(w.y >> 16, w.w >> 16, thr) << sh;
+        }
+      }
+      uint32_t keep[4];
+#pragma unroll
+      for (int wd = 0; wd < 4; ++wd) {
+        auto pick = [&](int k) { return k == 0 ? a0[wd] : k == 1 ? a1[wd] : k == 2 ? a2[wd] : a3[wd]; };
+        uint32_t kw = pick(r);
+        kw |= __shfl_xor_sync(0xffffffffu, pick(r ^ 1), 1);
+        kw |= __shfl_xor_sync(0xffffffffu, pick(r ^ 2), 2);
+        kw |= __shfl_xor_sync(0xffffffffu, pick(r ^ 3), 3);
+        keep[wd] = kw;
+      }
+      ring[slot * kT + rt] = make_uint4(keep[0], keep[1], keep[2], keep[3]);
+      mbar_arrive(bar(L::kBarKeepFull + slot));
+    }
   } else {
+    if constexpr (DROP) regs_increase<kRegsElem>();
     // ------------------------------------------------------------------ elementwise: one key row per thread
     const int wq = warp;
     const int jrow = wq * 32 + lane;
@@ -327,42 +389,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < nt; ++t) {
       const int buf = t & 1;
       const int i0 = (mstart + t % per_head) * kT;
-      uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit cc = (query i0 + cc, this key) kept
-      if constexpr (DROP) {
-        // drawn before the scores arrive, four independent Philox calls at a time.  Lanes 4m ..
-        // 4m + 3 hold the four keys of one key quad, which share every call: each lane makes the
-        // calls of every fourth query pair, which give two bits (the pair's queries) for each key
-        // of the quad, and the lanes swap them (lane ^ 1, ^ 2, ^ 3)
-        const uint32_t bh = (uint32_t)(b * p.Hq + hk * G + t / per_head), jq = (uint32_t)key >> 2;
-        const int r = key & 3;  // == lane & 3
-        const uint32_t thr = p.drop.thr;
-        uint32_t a0[4] = {0u, 0u, 0u, 0u}, a1[4] = {0u, 0u, 0u, 0u};  // bits of keys 4 jq + k at this
-        uint32_t a2[4] = {0u, 0u, 0u, 0u}, a3[4] = {0u, 0u, 0u, 0u};  // lane's query pairs, by word
-#pragma unroll 1
-        for (int t2 = 0; t2 < 4; ++t2) {
-#pragma unroll
-          for (int wd = 0; wd < 4; ++wd) {
-            // the call of the 2 x 4 block (queries i0 + cc, + 1) x (keys 4 jq .. 4 jq + 3)
-            const int cc = 32 * wd + 8 * t2 + 2 * r;
-            const uint4 w = philox4x32_10(jq, (uint32_t)(i0 + cc) >> 1, bh, p.drop.offset, p.drop.seed_lo,
-                                          p.drop.seed_hi);
-            const int sh = cc & 31;
-            a0[wd] |= keep_pair(w.x & 0xFFFFu, w.z & 0xFFFFu, thr) << sh;
-            a1[wd] |= keep_pair(w.x >> 16, w.z >> 16, thr) << sh;
-            a2[wd] |= keep_pair(w.y & 0xFFFFu, w.w & 0xFFFFu, thr) << sh;
-            a3[wd] |= keep_pair(w.y >> 16, w.w >> 16, thr) << sh;
-          }
-        }
-#pragma unroll
-        for (int wd = 0; wd < 4; ++wd) {
-          auto pick = [&](int k) { return k == 0 ? a0[wd] : k == 1 ? a1[wd] : k == 2 ? a2[wd] : a3[wd]; };
-          uint32_t kw = pick(r);
-          kw |= __shfl_xor_sync(0xffffffffu, pick(r ^ 1), 1);
-          kw |= __shfl_xor_sync(0xffffffffu, pick(r ^ 2), 2);
-          kw |= __shfl_xor_sync(0xffffffffu, pick(r ^ 3), 3);
-          keep[wd] = kw;
-        }
-      }
       float nl = 0.f, nd = 0.f;
       if (t + 1 < nt) fetch(t + 1, nl, nd);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarLse + buf), (t >> 1) & 1, abort_flag, p.status));
@@ -385,6 +411,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < kT; ++cc)
           if (cc < lim) pv[cc] = 0.f;
+      }
+      uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit cc = (query i0 + cc, this key) kept
+      if constexpr (DROP) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarKeepFull + (t & 1)), (t >> 1) & 1, abort_flag, p.status));
+        if (!ok) break;
+        const uint4 kq = reinterpret_cast<const uint4*>(gb + L::kOffKeep)[(t & 1) * kT + jrow];
+        keep[0] = kq.x;
+        keep[1] = kq.y;
+        keep[2] = kq.z;
+        keep[3] = kq.w;
+        mbar_arrive(bar(L::kBarKeepEmpty + (t & 1)));
       }
       {
         auto pd = [&](int c) { return DROP && !((keep[c >> 5] >> (c & 31)) & 1u) ? 0.f : pv[c]; };
@@ -714,12 +751,13 @@ template <typename T, int D, bool CAUSAL>
 cudaError_t launch_dkdv(const BwdArgs& a, cudaStream_t s) {
   Maps m;
   if (!make_maps(m, a, true, false)) return cudaErrorInvalidValue;
-  auto kern = a.drop_p > 0.f ? bwd_dkdv_sm100_kernel<T, D, CAUSAL, true> : bwd_dkdv_sm100_kernel<T, D, CAUSAL, false>;
+  const bool drop = a.drop_p > 0.f;
+  auto kern = drop ? bwd_dkdv_sm100_kernel<T, D, CAUSAL, true> : bwd_dkdv_sm100_kernel<T, D, CAUSAL, false>;
   const int smem = DkdvSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.Hkv, (a.Nk + kT - 1) / kT, a.B);
-  kern<<<grid, kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, m.dk, m.dv, params(a, a.dk, a.dv));
+  kern<<<grid, drop ? kThreadsDrop : kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, m.dk, m.dv, params(a, a.dk, a.dv));
   return cudaGetLastError();
 }
 
