@@ -484,17 +484,21 @@ __global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
 // ===========================================================================
 // dQ
 // ===========================================================================
-template <int D>
+template <int D, bool DROP>
 struct DqSmem {
   static constexpr int kTile = (D / 64) * kPanel;
+  static constexpr int kVStages = DROP ? 1 : 2;  // with dropout one V stage makes room for the keep ring
   static constexpr int kOffQ = 0;
   static constexpr int kOffDO = kTile;
   static constexpr int kOffK = 2 * kTile;  // 3 stages
-  static constexpr int kOffV = 5 * kTile;  // 2 stages
-  static constexpr int kOffBar = 7 * kTile;
-  // kBarOut: the elementwise threads have staged dQ (in the free Q buffer)
+  static constexpr int kOffV = 5 * kTile;  // kVStages stages
+  static constexpr int kOffKeep = kOffV + kVStages * kTile;  // dropout: [2][128 rows] x 128 keep bits
+  static constexpr int kOffBar = kOffKeep + (DROP ? 2 * kT * 16 : 0);
+  // kBarOut: the elementwise threads have staged dQ (in the free Q buffer);
+  // kBarKeepFull / kBarKeepEmpty: a slot of the keep-bit ring written / read
   enum { kBarQ = 0, kBarKFull = 1, kBarKEmpty = 4, kBarVFull = 7, kBarVEmpty = 9, kBarS = 11, kBarDP = 13,
-         kBarDS = 14, kBarDone = 15, kBarDrain = 16, kBarOut = 17, kNumBars = 18 };
+         kBarDS = 14, kBarDone = 15, kBarDrain = 16, kBarOut = 17, kBarKeepFull = 18, kBarKeepEmpty = 20,
+         kNumBars = 22 };
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmem + 4;
   static constexpr int kBytes = kOffAbort + 4 + 1024;
@@ -504,11 +508,11 @@ __host__ __device__ constexpr uint32_t col_s(int buf) { return 128u * buf; }
 constexpr uint32_t kColDP = 256, kColDQ = 384;
 
 template <typename T, int D, bool CAUSAL, bool DROP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
     bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                         const __grid_constant__ CUtensorMap tmDQ, Params p) {
-  using L = DqSmem<D>;
+  using L = DqSmem<D, DROP>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
@@ -527,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n = (n_end + kT - 1) / kT;
 
   if (tid == 0) {
-    for (int i = 0; i < L::kNumBars; ++i) mbar_init(bar(i), (i == L::kBarDS || i == L::kBarOut) ? kT : 1);
+    for (int i = 0; i < L::kNumBars; ++i) mbar_init(bar(i), (i == L::kBarDS || i >= L::kBarOut) ? kT : 1);
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -547,10 +551,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(gb + L::kOffTmem);
 
-  if (warp == kWarpLoad) {
+  if (warp >= 4 && warp < 8) {
+   if constexpr (DROP) regs_decrease<kRegsCtrl>();
+   if (warp == kWarpLoad) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int last_k[3] = {-1, -1, -1}, last_v[2] = {-1, -1};
+      constexpr int VS = L::kVStages;
       mbar_expect_tx(bar(L::kBarQ), 2 * L::kTile);
 #pragma unroll
       for (int pn = 0; pn < D / 64; ++pn) {
@@ -558,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(sb + L::kOffDO + pn * kPanel, &tmDO, bar(L::kBarQ), 64 * pn, h, m0, b);
       }
       for (int j = 0; j < n; ++j) {
-        const int ks = j % 3, ku = j / 3, vs = j & 1, vu = j >> 1;
+        const int ks = j % 3, ku = j / 3, vs = j % VS, vu = j / VS;
         if (ku > 0 && !mbar_wait(bar(L::kBarKEmpty + ks), (ku - 1) & 1, abort_flag, p.status)) break;
         mbar_expect_tx(bar(L::kBarKFull + ks), L::kTile);
 #pragma unroll
@@ -578,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         wait_drain(bar(L::kBarQ), 0, p.status);
         for (int s3 = 0; s3 < 3; ++s3)
           if (last_k[s3] >= 0) wait_drain(bar(L::kBarKFull + s3), last_k[s3] & 1, p.status);
-        for (int s2 = 0; s2 < 2; ++s2)
+        for (int s2 = 0; s2 < VS; ++s2)
           if (last_v[s2] >= 0) wait_drain(bar(L::kBarVFull + s2), last_v[s2] & 1, p.status);
       }
     }
@@ -598,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       const uint32_t sQ = sb + L::kOffQ, sDO = sb + L::kOffDO;
       auto sK = [&](int j) { return sb + L::kOffK + (j % 3) * L::kTile; };
-      auto sV = [&](int j) { return sb + L::kOffV + (j & 1) * L::kTile; };
+      auto sV = [&](int j) { return sb + L::kOffV + (j % L::kVStages) * L::kTile; };
       auto issue_s = [&](int j) -> bool {
         if (!mbar_wait(bar(L::kBarKFull + j % 3), (j / 3) & 1, abort_flag, p.status)) return false;
         tc_fence_after();
@@ -607,11 +614,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       auto issue_dp = [&](int j) -> bool {
-        if (!mbar_wait(bar(L::kBarVFull + (j & 1)), (j >> 1) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(bar(L::kBarVFull + j % L::kVStages), (j / L::kVStages) & 1, abort_flag, p.status)) return false;
         tc_fence_after();
         kmajor(kColDP, sDO, sV(j));
         mma_commit(bar(L::kBarDP));
-        mma_commit(bar(L::kBarVEmpty + (j & 1)));
+        mma_commit(bar(L::kBarVEmpty + j % L::kVStages));
         return true;
       };
       bool ok = mbar_wait(bar(L::kBarQ), 0, abort_flag, p.status);
@@ -635,7 +642,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar(L::kBarDrain));
       wait_drain(bar(L::kBarDrain), 0, p.status);
     }
+  }
+  } else if (DROP && warp >= 8) {
+    if constexpr (DROP) regs_decrease<kRegsRng>();
+    // ------------------------------------------------------------------ keep bits (dropout)
+    // thread rt draws the keep bits of query row m0 + rt for every key tile into ring slot j & 1.
+    // Lanes 2m and 2m + 1 hold one query pair: each makes the calls of every other key quad and
+    // hands the other row's bits to lane ^ 1; four independent calls are in flight at a time.
+    const int rt = tid - 256;
+    const int row = m0 + rt;
+    const uint32_t bh = (uint32_t)(b * p.Hq + h), rh = (uint32_t)row >> 1;
+    const int e = row & 1;  // == lane & 1
+    uint4* ring = reinterpret_cast<uint4*>(gb + L::kOffKeep);
+    for (int j = 0; j < n; ++j) {
+      const int slot = j & 1;
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar(L::kBarKeepEmpty + slot), ((j >> 1) - 1) & 1,
+                                                       abort_flag, p.status)))
+        break;
+      const int kb = j * kT;
+      uint32_t own[4] = {0u, 0u, 0u, 0u}, other[4] = {0u, 0u, 0u, 0u};
+#pragma unroll 1
+      for (int t2 = 0; t2 < 4; ++t2) {
+#pragma unroll
+        for (int wd = 0; wd < 4; ++wd) {
+          const int cc = 32 * wd + 8 * t2 + 4 * e;  // keys kb + cc .. cc + 3
+          const uint4 w = philox4x32_10((uint32_t)(kb + cc) >> 2, rh, bh, p.drop.offset, p.drop.seed_lo,
+                                        p.drop.seed_hi);
+          const uint32_t even = keep_quad(w.x, w.y, p.drop.thr), odd = keep_quad(w.z, w.w, p.drop.thr);
+          own[wd] |= (e ? odd : even) << (cc & 31);
+          other[wd] |= (e ? even : odd) << (cc & 31);
+        }
+      }
+      uint32_t keep[4];
+#pragma unroll
+      for (int wd = 0; wd < 4; ++wd) keep[wd] = own[wd] | __shfl_xor_sync(0xffffffffu, other[wd], 1);
+      ring[slot * kT + rt] = make_uint4(keep[0], keep[1], keep[2], keep[3]);
+      mbar_arrive(bar(L::kBarKeepFull + slot));
+    }
   } else {
+    if constexpr (DROP) regs_increase<kRegsElem>();
     // ------------------------------------------------------------------ elementwise: one query row per thread
     const int wq = warp;
     const int row = m0 + wq * 32 + lane;
@@ -648,29 +693,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < n; ++j) {
       const uint32_t tS = tbase + lane_off + col_s(j & 1);
       const int kb = j * kT;
-      uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit cc = (this query, key kb + cc) kept
-      if constexpr (DROP) {
-        // drawn before the scores arrive, four independent Philox calls at a time.  Lanes 2m and
-        // 2m + 1 hold one query pair: each makes the calls of every other key quad and hands the
-        // other row's bits to lane ^ 1
-        const uint32_t bh = (uint32_t)(b * p.Hq + h), rh = (uint32_t)row >> 1;
-        const int e = row & 1;  // == lane & 1
-        uint32_t own[4] = {0u, 0u, 0u, 0u}, other[4] = {0u, 0u, 0u, 0u};
-#pragma unroll 1
-        for (int t2 = 0; t2 < 4; ++t2) {
-#pragma unroll
-          for (int wd = 0; wd < 4; ++wd) {
-            const int cc = 32 * wd + 8 * t2 + 4 * e;  // keys kb + cc .. cc + 3
-            const uint4 w = philox4x32_10((uint32_t)(kb + cc) >> 2, rh, bh, p.drop.offset, p.drop.seed_lo,
-                                          p.drop.seed_hi);
-            const uint32_t even = keep_quad(w.x, w.y, p.drop.thr), odd = keep_quad(w.z, w.w, p.drop.thr);
-            own[wd] |= (e ? odd : even) << (cc & 31);
-            other[wd] |= (e ? even : odd) << (cc & 31);
-          }
-        }
-#pragma unroll
-        for (int wd = 0; wd < 4; ++wd) keep[wd] = own[wd] | __shfl_xor_sync(0xffffffffu, other[wd], 1);
-      }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + (j & 1)), (j >> 1) & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
@@ -693,6 +715,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), j & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
+      uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit cc = (this query, key kb + cc) kept
+      if constexpr (DROP) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarKeepFull + (j & 1)), (j >> 1) & 1, abort_flag, p.status));
+        if (!ok) break;
+        const uint4 kq = reinterpret_cast<const uint4*>(gb + L::kOffKeep)[(j & 1) * kT + wq * 32 + lane];
+        keep[0] = kq.x;
+        keep[1] = kq.y;
+        keep[2] = kq.z;
+        keep[3] = kq.w;
+        mbar_arrive(bar(L::kBarKeepEmpty + (j & 1)));
+      }
       write_ds<T, false, DROP>(tbase + lane_off + kColDP, tS, pv, nullptr, ndrow, keep, p.drop.inv_keep);
       tmem_wait_st();
       tc_fence_before();
@@ -765,12 +798,13 @@ template <typename T, int D, bool CAUSAL>
 cudaError_t launch_dq(const BwdArgs& a, cudaStream_t s) {
   Maps m;
   if (!make_maps(m, a, false, true)) return cudaErrorInvalidValue;
-  auto kern = a.drop_p > 0.f ? bwd_dq_sm100_kernel<T, D, CAUSAL, true> : bwd_dq_sm100_kernel<T, D, CAUSAL, false>;
-  const int smem = DqSmem<D>::kBytes;
+  const bool drop = a.drop_p > 0.f;
+  auto kern = drop ? bwd_dq_sm100_kernel<T, D, CAUSAL, true> : bwd_dq_sm100_kernel<T, D, CAUSAL, false>;
+  const int smem = drop ? DqSmem<D, true>::kBytes : DqSmem<D, false>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.Hq, (a.Nq + kT - 1) / kT, a.B);
-  kern<<<grid, kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, m.dq, params(a, a.dq, nullptr));
+  kern<<<grid, drop ? kThreadsDrop : kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, m.dq, params(a, a.dq, nullptr));
   return cudaGetLastError();
 }
 
