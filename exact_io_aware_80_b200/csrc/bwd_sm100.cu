@@ -26,8 +26,11 @@
 //   exponentials of one tile overlap the MMAs of the next.
 //
 // With DROP both kernels regenerate the forward pass's dropout mask (Philox
-// words from the same counters, common.cuh): dV uses P * M, and dS =
-// P * (M * dP / (1 - p) - D); dV is scaled by 1 / (1 - p) when stored.
+// values from the same counters, common.cuh): dV uses P * M, and dS =
+// P * (M * dP / (1 - p) - D); dV is scaled by 1 / (1 - p) when stored.  A
+// third warpgroup (384 threads, setmaxnreg split) draws each tile's keep bits
+// into a two-slot shared-memory ring one tile ahead of the elementwise warps;
+// the dQ kernel's DROP variant keeps one V stage to make room for it.
 //
 // Every mbarrier wait is bounded (sm100.cuh) and the roles drain in-flight
 // copies and MMAs before tensor memory is released.
