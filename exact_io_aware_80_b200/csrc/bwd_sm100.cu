@@ -778,6 +778,15 @@ bool make_maps(Maps& m, const BwdArgs& a, bool kv_out, bool q_out) {
   return ok;
 }
 
+// The dropout kernels' register split assumes the launch register count it was sized against;
+// a kernel compiled with fewer would wait forever in setmaxnreg.inc, so it is not launched.
+template <typename K>
+bool split_fits(K kern) {
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return false;
+  return fa.numRegs * kThreadsDrop >= 128 * (kRegsElem + kRegsCtrl + kRegsRng);
+}
+
 Params params(const BwdArgs& a, void* out0, void* out1) {
   return Params{a.lse,  a.dvec,      out0,  out1, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, a.scale, a.scale * kLog2e, a.status,
                 Dropout{a.drop_thr, a.drop_inv_keep, a.seed_lo, a.seed_hi, a.drop_offset}};
@@ -792,6 +801,7 @@ cudaError_t launch_dkdv(const BwdArgs& a, cudaStream_t s) {
   const int smem = DkdvSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  if (drop && !split_fits(kern)) return cudaErrorInvalidConfiguration;
   dim3 grid(a.Hkv, (a.Nk + kT - 1) / kT, a.B);
   kern<<<grid, drop ? kThreadsDrop : kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, m.dk, m.dv, params(a, a.dk, a.dv));
   return cudaGetLastError();
@@ -806,6 +816,7 @@ cudaError_t launch_dq(const BwdArgs& a, cudaStream_t s) {
   const int smem = drop ? DqSmem<D, true>::kBytes : DqSmem<D, false>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  if (drop && !split_fits(kern)) return cudaErrorInvalidConfiguration;
   dim3 grid(a.Hq, (a.Nq + kT - 1) / kT, a.B);
   kern<<<grid, drop ? kThreadsDrop : kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, m.dq, params(a, a.dq, nullptr));
   return cudaGetLastError();
