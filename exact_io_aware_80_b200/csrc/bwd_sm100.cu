@@ -25,6 +25,9 @@
 //   dP = dO V^T, then dQ += dS K; S for tile j+2 is queued behind dQ_j so the
 //   exponentials of one tile overlap the MMAs of the next.
 //
+// Both kernels write their outputs through shared memory (buffers that are
+// free once the last MMA has run) and TMA stores.
+//
 // With DROP both kernels regenerate the forward pass's dropout mask (Philox
 // values from the same counters, common.cuh): dV uses P * M, and dS =
 // P * (M * dP / (1 - p) - D); dV is scaled by 1 / (1 - p) when stored.  A
@@ -157,7 +160,7 @@ struct DkdvSmem {
   static constexpr int kOffD = kOffLse + 2 * kT * 4;
   static constexpr int kOffKeep = kOffD + 2 * kT * 4;  // dropout: [2][128 keys] x 128 keep bits
   static constexpr int kOffBar = kOffKeep + 2 * kT * 16;
-  // kBarOut: the elementwise threads have staged dK and dV (in the free Q / dO buffers);
+  // kBarOut: the elementwise threads have staged dK and dV (in the two free Q stages);
   // kBarKeepFull / kBarKeepEmpty: a slot of the keep-bit ring written / read
   enum { kBarKV = 0, kBarQFull = 1, kBarQEmpty = 3, kBarS = 5, kBarDP = 6, kBarP = 7, kBarDS = 8, kBarDone = 9,
          kBarDrain = 10, kBarLse = 11, kBarOut = 13, kBarKeepFull = 14, kBarKeepEmpty = 16, kNumBars = 18 };
