@@ -276,6 +276,10 @@ def run_ours(args):
                                                          world, peaks, peaks_kind)
     drop = None if args.no_dropout else run_dropout(args, torch, fa, _lib, w, q, k, v, do, dev, stream, world)
     ringl = None if args.no_ring else run_ring_local(args, torch, w, q, k, v, dev, stream, world)
+    mha = None if args.no_mha else run_mha_prefill(args, torch, fa, _lib, workloads, dev, stream, world, peaks,
+                                                   peaks_kind)
+    longc = None if args.no_long else run_long_context(args, torch, fa, _lib, workloads, dev, stream, world, peaks,
+                                                       peaks_kind)
     e2e = run_e2e(args, torch, fa, w, q, k, v, do, dev, stream, world, F) if not args.no_e2e else None
 
     cpu = None
@@ -303,6 +307,8 @@ def run_ours(args):
         "blocksparse": sparse,
         "dropout": drop,
         "ring_local": ringl,
+        "mha_prefill": mha,
+        "long_context": longc,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -565,6 +571,133 @@ def run_ring_local(args, torch, w, q, k, v, dev, stream, world):
             "gpu_launches": K * (W * (W + 1) - 1)}  # W(W+1)/2 forward launches, one merge fewer (rank 0 copies)
 
 
+def _peak_for(peaks, region_ms):
+    key = "bf16_tflops_sustained" if region_ms >= 2000 else "bf16_tflops"
+    return float(peaks.get(key, FALLBACK_PEAKS[key])), key
+
+
+def run_mha_prefill(args, torch, fa, _lib, workloads, dev, stream, world, peaks, peaks_kind):
+    """MHA prefill forward, B=4, H=16, N=2048, d=128 bf16, causal and non-causal.  Its four tensors
+    (Q, K, V, O: 128 MiB) are about the size of L2, so L2 is flushed (a 256 MiB write) before every
+    timed launch and each launch is timed alone with CUDA events on the launching stream."""
+    w = workloads.get(2)
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.Nq, w.d
+    q, k, v = workloads.workload_inputs(w, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, N, device=dev, dtype=torch.float32)
+    flush = torch.empty(256 << 20, device=dev, dtype=torch.uint8)
+    sh = stream.cuda_stream
+    out = {"workload": f"MHA prefill forward: B={B} Hq=Hkv={Hq} Nq=Nk={N} d={d} bf16",
+           "l2": "flushed before every timed launch (256 MiB write, outside the timed events)"}
+    total_ms = 0.0
+    for causal in (False, True):
+        def launch():
+            _lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, N, d,
+                        int(causal), w.scale, _lib.FA_BF16, sh)
+
+        for _ in range(args.warmup):
+            launch()
+        K = args.steps
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        barrier(torch, world)
+        torch.cuda.synchronize(dev)
+        for e0, e1 in evs:
+            flush.fill_(1)
+            e0.record(stream)
+            launch()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(torch, world)
+        if fa.device_status() != 0:
+            raise RuntimeError("kernel status word set during the MHA prefill section")
+        ms = max_over_ranks(torch, world, statistics.fmean(e0.elapsed_time(e1) for e0, e1 in evs))
+        total_ms += ms * K
+        F = attn_flops(B, Hq, N, N, d, causal)
+        ach = F / (ms * 1e-3) / 1e12
+        peak, key = _peak_for(peaks, ms * K)
+        out["causal" if causal else "noncausal"] = {
+            "ms": round(ms, 4), "value": round(world * ach, 1), "unit": "TFLOP/s",
+            "frac_of_datasheet_2250": round(ach / DENSE_BF16_DATASHEET_TFLOPS, 4),
+            "roofline": {"bound": "tensor", "kernel": "fwd_sm100_kernel", "achieved": round(ach, 1), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                         "peak_source": f"{peaks_kind} {key}", "algorithmic_flops_per_launch": F},
+            "gpu_launches": K}
+    return out
+
+
+def run_long_context(args, torch, fa, _lib, workloads, dev, stream, world, peaks, peaks_kind):
+    """Long-context GQA step, B=1, Hq=32, Hkv=8, N=16384, d=128 bf16 causal: forward + the three
+    backward launches, timed per launch like the headline step (each step touches ~650 MiB, more
+    than L2, so no flush)."""
+    w = workloads.get(4)
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.Nq, w.d
+    q, k, v, do = workloads.workload_inputs(w, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, N, device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_workspace_bytes(B, Hq, N), device=dev, dtype=torch.uint8)
+    sh = stream.cuda_stream
+    dt = _lib.FA_BF16
+    bargs = [t.data_ptr() for t in (q, k, v, o, do, lse, dq, dk, dv, ws)] + [B, Hq, Hkv, N, N, d, 1, w.scale, dt, sh]
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        _lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, N, d, 1,
+                    w.scale, dt, sh)
+        if ev:
+            ev[1].record(stream)
+        _lib.fa_bwd_preprocess(*bargs)
+        if ev:
+            ev[2].record(stream)
+        _lib.fa_bwd_dkdv(*bargs)
+        if ev:
+            ev[3].record(stream)
+        _lib.fa_bwd_dq(*bargs)
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    K = max(3, args.steps // 2)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    barrier(torch, world)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(torch, world)
+    if fa.device_status() != 0:
+        raise RuntimeError("kernel status word set during the long-context section")
+    ms_total = t0.elapsed_time(t1)
+    ms = max_over_ranks(torch, world, ms_total) / K
+    per = {name: statistics.fmean(e[j].elapsed_time(e[j + 1]) for e in evs)
+           for j, name in enumerate(("fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"))}
+    F = attn_flops(B, Hq, N, N, d, True)
+    bwd_ms = per["bwd_preprocess"] + per["bwd_dkdv"] + per["bwd_dq"]
+    peak, key = _peak_for(peaks, ms_total)
+    kflops = {"fwd": F, "bwd_dkdv": 2.0 * F, "bwd_dq": 1.5 * F}
+    dom = max(kflops, key=lambda n: per[n])
+    kname = {"fwd": "fwd_sm100_kernel", "bwd_dkdv": "bwd_dkdv_sm100_kernel", "bwd_dq": "bwd_dq_sm100_kernel"}[dom]
+    ach = kflops[dom] / (per[dom] * 1e-3) / 1e12
+    fwd_t, bwd_t = F / (per["fwd"] * 1e-3) / 1e12, 2.5 * F / (bwd_ms * 1e-3) / 1e12
+    return {"workload": f"long-context GQA step: fwd+bwd, B={B} Hq={Hq} Hkv={Hkv} Nq=Nk={N} d={d} causal bf16",
+            "ms_per_step": round(ms, 4), "value": round(world * 3.5 * F / (ms * 1e-3) / 1e12, 1), "unit": "TFLOP/s",
+            "fwd_ms": round(per["fwd"], 4), "fwd_tflops": round(fwd_t, 1),
+            "fwd_frac_of_datasheet_2250": round(fwd_t / DENSE_BF16_DATASHEET_TFLOPS, 4),
+            "bwd_ms": round(bwd_ms, 4), "bwd_tflops": round(bwd_t, 1),
+            "bwd_frac_of_datasheet_2250": round(bwd_t / DENSE_BF16_DATASHEET_TFLOPS, 4),
+            "per_kernel_ms": {kk: round(vv, 4) for kk, vv in per.items()},
+            "roofline": {"bound": "tensor", "kernel": kname, "achieved": round(ach, 1), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                         "peak_source": f"{peaks_kind} {key}", "algorithmic_flops_per_launch": kflops[dom],
+                         "avg_launch_ms": round(per[dom], 4)},
+            "gpu_launches": 4 * K}
+
+
 def run_e2e(args, torch, fa, w, q, k, v, do, dev, stream, world, F):
     """Same step through the public Python API with host buffers: every step uploads q, k, v, dO from
     pinned host memory, runs the forward and backward, and downloads dQ, dK, dV, all inside the timed
@@ -726,6 +859,8 @@ def main():
     ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse section (profiling runs)")
     ap.add_argument("--no-dropout", action="store_true", help="skip the dropout section (profiling runs)")
     ap.add_argument("--no-ring", action="store_true", help="skip the one-GPU ring-attention section")
+    ap.add_argument("--no-mha", action="store_true", help="skip the MHA prefill section (B=4 H=16 N=2048)")
+    ap.add_argument("--no-long", action="store_true", help="skip the long-context section (N=16384)")
     ap.add_argument("--decode-b", type=int, default=0,
                     help="override B of the decode workload (profiling runs on a smaller case)")
     ap.add_argument("--seq", type=int, default=0,

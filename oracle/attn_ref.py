@@ -31,7 +31,7 @@ Sources (page title, section):
 * smithlab guide, "FlashAttention 도입 체크리스트": causal is a flag and GQA is
   expressed by the KV-head count, with no K/V replication.
 
-Readings where the pages are silent (each is listed in the design doc too):
+Readings where the pages are silent:
 
 * layout BSHD: q, o, do, dq are [B, Nq, Hq, d]; k, v, dk, dv are
   [B, Nk, Hkv, d]; lse is [B, Hq, Nq];
@@ -70,7 +70,6 @@ __all__ = [
     "attention_flops",
     "lse_bytes",
     "eager_softmax_bytes",
-    "kv_cache_bytes",
     "brute_force_attention",
     "attention_bwd_partial",
 ]
@@ -432,10 +431,6 @@ def eager_softmax_bytes(B: int, Hq: int, Nq: int, Nk: int, layers: int = 1) -> i
     (smithlab guide, memory table)."""
     return B * Hq * Nq * Nk * 6 * layers
 
-
-def kv_cache_bytes(seqlens_k, Hkv: int, d: int, elem_bytes: int = 2) -> int:
-    """Bytes of K and V a decode step must read: sum_b Nk_b * Hkv * d * 2 tensors."""
-    return int(sum(int(n) for n in seqlens_k)) * Hkv * d * elem_bytes * 2
 
 
 def brute_force_attention(q, k, v, causal: bool, scale: float):

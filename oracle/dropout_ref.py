@@ -7,7 +7,7 @@ Sources: "FlashAttention 심층 분석" (ryotta.opik.net), section 2: dropout is
 of the steps the kernel fuses (scaling, masking, softmax, dropout, the P V
 product); section 4: the backward pass recomputes what it needs instead of
 storing it -- for dropout that means regenerating the same mask.  The pages
-name no generator and no keep rule.  Readings (listed in the design doc):
+name no generator and no keep rule.  Readings:
 
 * generator: Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, "Parallel
   random numbers: as easy as 1, 2, 3", SC 2011), written here from that
@@ -61,59 +61,89 @@ def keep_threshold(p: float) -> int:
     return min(int(np.floor(p * 65536.0)), 0xFFFF)
 
 
-def keep_mask(b: int, h: int, Hq: int, Nq: int, Nk: int, p: float, seed: int, offset: int) -> np.ndarray:
-    """Boolean [Nq, Nk]: True where (i, j) of head (b, h) is kept."""
-    i = np.arange(Nq, dtype=np.uint64)[:, None]
-    j = np.arange(Nk, dtype=np.uint64)[None, :]
-    ii, jj = np.broadcast_arrays(i, j)
-    words = philox4x32(jj >> np.uint64(2), ii >> np.uint64(1), np.full(ii.shape, b * Hq + h, np.uint64),
-                       np.full(ii.shape, offset, np.uint64), seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
-    e = (4 * (ii & np.uint64(1)) + (jj & np.uint64(3))).astype(np.int64)
-    w = np.choose(e >> 1, words)
-    value = (w >> (np.uint64(16) * (e & 1).astype(np.uint64))) & np.uint64(0xFFFF)
-    return value >= np.uint64(keep_threshold(p))
+def keep_mask(b: int, h: int, Hq: int, Nq: int, Nk: int, p: float, seed: int, offset: int, rows=None) -> np.ndarray:
+    """Boolean [Nq, Nk] (or [len(rows), Nk]): True where (i, j) of head (b, h) is kept.
+
+    One Philox call per 2 x 4 block of (query pair i >> 1, key quad j >> 2) that the
+    requested rows touch; element (i, j) reads 16-bit value e = 4 (i & 1) + (j & 3)
+    of its block's call (half e & 1 of word e >> 1).
+    """
+    rows = np.arange(Nq, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    pairs = np.unique(rows >> 1)
+    quads = np.arange((Nk + 3) // 4, dtype=np.int64)
+    pp, qq = np.meshgrid(pairs.astype(np.uint64), quads.astype(np.uint64), indexing="ij")
+    words = philox4x32(qq, pp, np.full(pp.shape, b * Hq + h, np.uint64), np.full(pp.shape, offset, np.uint64),
+                       seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
+    values = np.stack([((words[e >> 1] >> np.uint64(16 * (e & 1))) & np.uint64(0xFFFF)).astype(np.uint16)
+                       for e in range(8)])  # [8, pairs, quads]
+    j = np.arange(Nk, dtype=np.int64)
+    e = 4 * (rows & 1)[:, None] + (j & 3)[None, :]
+    value = values[e, np.searchsorted(pairs, rows >> 1)[:, None], (j >> 2)[None, :]]
+    return value >= keep_threshold(p)
 
 
-def attention_fwd_dropout(q, k, v, causal: bool, scale: float, p: float, seed: int, offset: int):
-    """O [B, Nq, Hq, d] and LSE [B, Hq, Nq] (fp64) with dropout on P."""
+def attention_fwd_dropout(q, k, v, causal: bool, scale: float, p: float, seed: int, offset: int, heads=None,
+                          row_chunk: int = 2048):
+    """O [B, Nq, Hq, d] and LSE [B, Hq, Nq] (fp64) with dropout on P.
+
+    ``heads`` optionally restricts the work to a list of (b, h_q) pairs (the other
+    outputs stay NaN).  Query rows are taken ``row_chunk`` at a time to bound
+    memory; every row's softmax still spans its whole score row, so the chunking
+    changes no value.
+    """
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, Nq, Nk, Hq, Hkv, d = _check_shapes(q, k, v)
     G = Hq // Hkv
     vis = visible_mask(Nq, Nk, causal)
-    O = np.empty((B, Nq, Hq, d))
-    LSE = np.empty((B, Hq, Nq))
-    for b in range(B):
-        for h in range(Hq):
-            S = scores(q[b, :, h, :], k[b, :, h // G, :], scale, vis)
+    O = np.full((B, Nq, Hq, d), np.nan)
+    LSE = np.full((B, Hq, Nq), np.nan)
+    todo = heads if heads is not None else [(b, h) for b in range(B) for h in range(Hq)]
+    for b, h in todo:
+        for i0 in range(0, Nq, row_chunk):
+            rows = np.arange(i0, min(i0 + row_chunk, Nq))
+            S = scores(q[b, rows, h, :], k[b, :, h // G, :], scale, vis[rows])
             P, lse = softmax_rows(S)
-            M = keep_mask(b, h, Hq, Nq, Nk, p, seed, offset)
-            O[b, :, h, :] = (P * M / (1.0 - p)) @ v[b, :, h // G, :]
-            LSE[b, h, :] = lse
+            M = keep_mask(b, h, Hq, Nq, Nk, p, seed, offset, rows)
+            O[b, rows, h, :] = (P * M / (1.0 - p)) @ v[b, :, h // G, :]
+            LSE[b, h, rows] = lse
     return O, LSE
 
 
-def attention_bwd_dropout(q, k, v, do, causal: bool, scale: float, p: float, seed: int, offset: int):
-    """dQ, dK, dV (fp64) of sum(dO * O) for the dropout forward above (same mask)."""
+def attention_bwd_dropout(q, k, v, do, causal: bool, scale: float, p: float, seed: int, offset: int, kv_heads=None,
+                          row_chunk: int = 2048):
+    """dQ, dK, dV (fp64) of sum(dO * O) for the dropout forward above (same mask).
+
+    ``kv_heads`` optionally restricts the work to a list of (b, h_kv) pairs (their
+    query heads' dQ and their own dK, dV; the rest stays NaN).  Query rows are
+    taken ``row_chunk`` at a time; dK and dV add up the chunks' contributions.
+    """
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     B, Nq, Nk, Hq, Hkv, d = _check_shapes(q, k, v)
     G = Hq // Hkv
     vis = visible_mask(Nq, Nk, causal)
-    dq = np.zeros_like(q)
-    dk = np.zeros_like(k)
-    dv = np.zeros_like(v)
+    dq = np.full_like(q, np.nan)
+    dk = np.full_like(k, np.nan)
+    dv = np.full_like(v, np.nan)
     r = 1.0 / (1.0 - p)
-    for b in range(B):
-        for h in range(Hq):
-            hk = h // G
-            S = scores(q[b, :, h, :], k[b, :, hk, :], scale, vis)
-            P, _ = softmax_rows(S)
-            M = keep_mask(b, h, Hq, Nq, Nk, p, seed, offset)
-            Pd = P * M * r
-            O = Pd @ v[b, :, hk, :]
-            dv[b, :, hk, :] += Pd.T @ do[b, :, h, :]
-            dP = M * r * (do[b, :, h, :] @ v[b, :, hk, :].T)
-            D = np.sum(do[b, :, h, :] * O, axis=1, keepdims=True)
-            dS = P * (dP - D)
-            dq[b, :, h, :] = scale * dS @ k[b, :, hk, :]
-            dk[b, :, hk, :] += scale * dS.T @ q[b, :, h, :]
+    todo = kv_heads if kv_heads is not None else [(b, hk) for b in range(B) for hk in range(Hkv)]
+    for b, hk in todo:
+        K, V = k[b, :, hk, :], v[b, :, hk, :]
+        dK = np.zeros((Nk, d))
+        dV = np.zeros((Nk, d))
+        for h in range(hk * G, (hk + 1) * G):
+            for i0 in range(0, Nq, row_chunk):
+                rows = np.arange(i0, min(i0 + row_chunk, Nq))
+                Q, dO = q[b, rows, h, :], do[b, rows, h, :]
+                P, _ = softmax_rows(scores(Q, K, scale, vis[rows]))
+                M = keep_mask(b, h, Hq, Nq, Nk, p, seed, offset, rows)
+                Pd = P * M * r
+                O = Pd @ V
+                dV += Pd.T @ dO
+                dP = M * r * (dO @ V.T)
+                D = np.sum(dO * O, axis=1, keepdims=True)
+                dS = P * (dP - D)
+                dq[b, rows, h, :] = scale * dS @ K
+                dK += scale * dS.T @ Q
+        dk[b, :, hk, :] = dK
+        dv[b, :, hk, :] = dV
     return dq, dk, dv

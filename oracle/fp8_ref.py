@@ -17,7 +17,7 @@ Sources (page title, section):
   2.6x lower error than a baseline FP8 attention).
 
 The pages name the technique but give no formats, scales or rotation.  The
-readings used here (each listed in the design doc):
+readings used here:
 
 * 8-bit format: E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits;
   largest finite 448, subnormals down to 2^-9, no infinities), conversion by
@@ -58,7 +58,6 @@ __all__ = [
     "dequantize_v",
     "attention_fp8_ref",
     "p_rounding_bound",
-    "fp8_flops",
 ]
 
 E4M3_MAX = 448.0
@@ -250,12 +249,6 @@ def p_rounding_bound(q8, q_scale, k8, k_scale, v8t, v_scale, Nk: int, causal: bo
     small = (w < 2.0 ** -6) & (w > 0)
     bound = (2.0 ** -4 * (w @ av) + 2.0 ** -10 * (small.astype(np.float64) @ av)) / np.where(l > 0, l, 1.0)
     return bound
-
-
-def fp8_flops(B: int, Hq: int, Nq: int, Nk: int, d: int, causal: bool) -> float:
-    """Nominal forward FLOPs, the same convention as the 16-bit forward."""
-    f = 4.0 * B * Hq * Nq * Nk * d
-    return f / 2 if causal else f
 
 
 def _self_check():  # pragma: no cover - a quick manual smoke

@@ -6,8 +6,7 @@ this module; it never imports the CUDA product package.
 Source: "FlashAttention-2 (KO)" (systems-analysis.info), "결과
 (FlashAttention-1)": extending the IO-aware kernel with a block-sparse pattern
 gives an approximate attention that is faster than earlier approximate
-methods.  The pages give neither the block size nor the mask format.  Readings
-(listed in DESIGN.md):
+methods.  The pages give neither the block size nor the mask format.  Readings:
 
 * the mask is a table of 128 x 128 blocks, ``block_mask[b, h, I, J]`` for query
   block I (rows 128 I .. 128 I + 127) and key block J, of shape

@@ -132,3 +132,37 @@ def test_planted_mistake_missing_rescale_is_caught():
         O, _ = dr.attention_fwd_dropout(q, k, v, False, 0.5, p, seed=1000 + s, offset=0)
         acc += O * (1 - p)  # what a kernel without the 1/(1-p) factor would return
     assert np.max(np.abs(acc / n - O0)) > 0.1
+
+
+def test_block_evaluated_mask_equals_one_call_per_element():
+    # brute force: one Philox call per (i, j) at the counter of its 2 x 4 block, value picked
+    # by e = 4 (i & 1) + (j & 3); odd sizes leave partial blocks at both edges
+    Nq, Nk, p, seed, off, b, h, Hq = 13, 23, 0.37, 0xA5A5_0F0F_1234_5678, 11, 1, 2, 3
+    M = dr.keep_mask(b, h, Hq, Nq, Nk, p, seed, off)
+    thr = dr.keep_threshold(p)
+    for i in range(Nq):
+        for j in range(Nk):
+            w = dr.philox4x32(np.array([j >> 2]), np.array([i >> 1]), np.array([b * Hq + h]), np.array([off]),
+                              seed & 0xFFFFFFFF, seed >> 32)
+            e = 4 * (i & 1) + (j & 3)
+            value = (int(w[e >> 1][0]) >> (16 * (e & 1))) & 0xFFFF
+            assert M[i, j] == (value >= thr), (i, j)
+    rows = [12, 0, 5, 6, 5]
+    np.testing.assert_array_equal(dr.keep_mask(b, h, Hq, Nq, Nk, p, seed, off, rows), M[rows])
+
+
+def test_sampled_heads_and_row_chunks_change_nothing():
+    q, k, v, do = rnd((2, 37, 4, 8), 21), rnd((2, 41, 2, 8), 22), rnd((2, 41, 2, 8), 23), rnd((2, 37, 4, 8), 24)
+    args = (True, 0.4, 0.2, 1234, 5)
+    O, L = dr.attention_fwd_dropout(q, k, v, *args)
+    O2, L2 = dr.attention_fwd_dropout(q, k, v, *args, heads=[(1, 3), (0, 0)], row_chunk=6)
+    for b, h in [(1, 3), (0, 0)]:
+        np.testing.assert_allclose(O2[b, :, h], O[b, :, h], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(L2[b, h], L[b, h], rtol=1e-12, atol=1e-14)
+    assert np.isnan(O2[0, :, 1]).all()
+    g = dr.attention_bwd_dropout(q, k, v, do, *args)
+    g2 = dr.attention_bwd_dropout(q, k, v, do, *args, kv_heads=[(1, 1)], row_chunk=7)
+    np.testing.assert_allclose(g2[0][1, :, 2:4], g[0][1, :, 2:4], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(g2[1][1, :, 1], g[1][1, :, 1], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(g2[2][1, :, 1], g[2][1, :, 1], rtol=1e-11, atol=1e-13)
+    assert np.isnan(g2[1][0]).all()

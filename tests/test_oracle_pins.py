@@ -352,10 +352,6 @@ def test_flop_convention_cost_table():
             assert usd == pytest.approx(row[n], abs=0.051), setup
 
 
-def test_kv_cache_bytes():
-    assert oracle.kv_cache_bytes([32768] * 2, 8, 128) == 2 * 32768 * 8 * 128 * 2 * 2
-
-
 # ---------------------------------------------------------------------------
 # planted mistakes: a copy of the oracle with one plausible error must fail a pin
 # ---------------------------------------------------------------------------
