@@ -406,9 +406,9 @@ def run_fp8(args, torch, fa, _lib, workloads, w, q, k, v, dev, stream, world, pe
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        _lib.fa_fp8_quantize_qk(q.data_ptr(), q8.data_ptr(), qs.data_ptr(), signs.data_ptr(), B, Hq, N, d, dt, sh)
-        _lib.fa_fp8_quantize_qk(k.data_ptr(), k8.data_ptr(), ks.data_ptr(), signs.data_ptr(), B, Hkv, N, d, dt, sh)
-        _lib.fa_fp8_quantize_v(v.data_ptr(), v8t.data_ptr(), vs.data_ptr(), vws.data_ptr(), B, Hkv, N, d, dt, sh)
+        _lib.fa_fp8_quantize_qkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), q8.data_ptr(), k8.data_ptr(), v8t.data_ptr(),
+                                 qs.data_ptr(), ks.data_ptr(), vs.data_ptr(), signs.data_ptr(), vws.data_ptr(), B, Hq,
+                                 Hkv, N, N, d, dt, sh)
         if ev:
             ev[1].record(stream)
         _lib.fa_fwd_fp8(q8.data_ptr(), qs.data_ptr(), k8.data_ptr(), ks.data_ptr(), v8t.data_ptr(), vs.data_ptr(),
@@ -438,14 +438,22 @@ def run_fp8(args, torch, fa, _lib, workloads, w, q, k, v, dev, stream, world, pe
     key = "bf16_tflops_sustained" if ms * K >= 2000 else "bf16_tflops"
     peak = 2.0 * float(peaks.get(key, FALLBACK_PEAKS[key]))  # e4m3 dense rate = 2x bf16 (nominal ratio)
     ach = F / (fwd_ms * 1e-3) / 1e12
+    # quantizers: Q, K read once, V twice (amax, then encode), codes written once
+    qbytes = (2 * (q.numel() + k.numel() + 2 * v.numel()) + q.numel() + k.numel() + v8t.numel() +
+              4 * (qs.numel() + ks.numel() + vs.numel()))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     return {"workload": f"FP8 (E4M3) forward, Q/K rotated: B={B} Hq={Hq} Hkv={Hkv} N={N} d={d} causal, bf16 in/out",
             "ms_per_step": round(ms, 4), "quantize_ms": round(quant_ms, 4), "fwd_ms": round(fwd_ms, 4),
             "fwd_tflops": round(ach, 1), "value": round(world * F / (ms * 1e-3) / 1e12, 1), "unit": "TFLOP/s",
+            "quantize": {"bytes": qbytes, "gbs": round(qbytes / (quant_ms * 1e-3) / 1e9, 1),
+                         "frac_of_measured_hbm": round(qbytes / (quant_ms * 1e-3) / 1e9 / hbm, 4),
+                         "launches": 2, "traffic": traffic_for("quant_kernel + v_quant_kernel")},
             "roofline": {"bound": "tensor", "kernel": "fwd_sm100_kernel (F8)", "achieved": round(ach, 1),
-                         "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                         "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                         "traffic": traffic_for("fwd_sm100_kernel (F8)"),
                          "peak_source": f"{peaks_kind} {key} x 2 (nominal e4m3 / bf16 ratio)",
                          "algorithmic_flops_per_launch": F},
-            "gpu_launches": 5 * K}
+            "gpu_launches": 3 * K}
 
 
 def run_blocksparse(args, torch, fa, _lib, workloads, w, q, k, v, dev, stream, world, peaks, peaks_kind):
@@ -493,7 +501,8 @@ def run_blocksparse(args, torch, fa, _lib, workloads, w, q, k, v, dev, stream, w
             "density_vs_causal": round(F / dense, 4), "ms_per_step": round(ms, 4),
             "value": round(world * ach, 1), "unit": "TFLOP/s (visible pairs)",
             "roofline": {"bound": "tensor", "kernel": "fwd_sm100_kernel (SPARSE)", "achieved": round(ach, 1),
-                         "peak": peak, "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                         "peak": peak, "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                         "traffic": traffic_for("fwd_sm100_kernel (SPARSE)"),
                          "peak_source": f"{peaks_kind} {key}", "algorithmic_flops_per_launch": F},
             "gpu_launches": K}
 

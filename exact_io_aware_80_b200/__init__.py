@@ -16,14 +16,16 @@ import math
 from . import _lib
 from ._lib import (FAError, fa_bwd, fa_bwd_dkdv, fa_bwd_dq, fa_bwd_preprocess, fa_bwd_workspace_bytes,  # noqa: F401
                    fa_decode_chunk, fa_decode_combine, fa_decode_num_splits, fa_decode_splitkv,
-                   fa_decode_workspace_bytes, fa_fp8_quantize_qk, fa_fp8_quantize_v, fa_fp8_v_workspace_bytes, fa_fwd,
+                   fa_decode_workspace_bytes, fa_fp8_quantize_qk, fa_fp8_quantize_qkv, fa_fp8_quantize_v,
+                   fa_fp8_v_workspace_bytes, fa_fwd,
                    fa_bwd_dropout, fa_fwd_blocksparse, fa_fwd_dropout, fa_fwd_fp8, fa_get_device_status, fa_version)
 
 __all__ = [
     "attention_fwd", "attention_bwd", "decode", "decode_splitkv", "decode_combine", "device_status",
     "fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq", "fa_decode_splitkv", "fa_decode_combine", "fa_decode_num_splits",
     "fa_decode_workspace_bytes", "fa_bwd_workspace_bytes", "fa_decode_chunk", "fa_get_device_status",
-    "fp8_quantize_qk", "fp8_quantize_v", "attention_fwd_fp8", "fa_fp8_quantize_qk", "fa_fp8_quantize_v",
+    "fp8_quantize_qk", "fp8_quantize_v", "fp8_quantize_qkv", "attention_fwd_fp8", "fa_fp8_quantize_qk",
+    "fa_fp8_quantize_qkv", "fa_fp8_quantize_v",
     "fa_fp8_v_workspace_bytes", "fa_fwd_fp8", "attention_fwd_blocksparse", "fa_fwd_blocksparse",
     "attention_fwd_dropout", "attention_bwd_dropout", "fa_fwd_dropout", "fa_bwd_dropout", "FAError",
 ]
@@ -145,6 +147,25 @@ def fp8_quantize_v(v):
     ws = torch.empty(fa_fp8_v_workspace_bytes(B, H, Nk), device=dev, dtype=torch.uint8)
     fa_fp8_quantize_v(v.data_ptr(), v8t.data_ptr(), sc.data_ptr(), ws.data_ptr(), B, H, Nk, d, _dt(v), _stream(dev))
     return v8t, sc
+
+
+def fp8_quantize_qkv(q, k, v, signs=None):
+    """Q, K, V quantized together (``fa_fp8_quantize_qkv``): (q8, q_scale, k8, k_scale, v8t, v_scale)."""
+    torch = _torch()
+    dev = _dev(q, k, v) if signs is None else _dev(q, k, v, signs)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    q8 = torch.empty(B, Nq, Hq, d, device=dev, dtype=torch.uint8)
+    k8 = torch.empty(B, Nk, Hkv, d, device=dev, dtype=torch.uint8)
+    v8t = torch.empty(B, Hkv, d, (Nk + 15) // 16 * 16, device=dev, dtype=torch.uint8)
+    qs = torch.empty(B, Hq, (Nq + 127) // 128, device=dev, dtype=torch.float32)
+    ks = torch.empty(B, Hkv, (Nk + 127) // 128, device=dev, dtype=torch.float32)
+    vs = torch.empty(B, Hkv, device=dev, dtype=torch.float32)
+    ws = torch.empty(fa_fp8_v_workspace_bytes(B, Hkv, Nk), device=dev, dtype=torch.uint8)
+    fa_fp8_quantize_qkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), q8.data_ptr(), k8.data_ptr(), v8t.data_ptr(),
+                        qs.data_ptr(), ks.data_ptr(), vs.data_ptr(), 0 if signs is None else signs.data_ptr(),
+                        ws.data_ptr(), B, Hq, Hkv, Nq, Nk, d, _dt(q), _stream(dev))
+    return q8, qs, k8, ks, v8t, vs
 
 
 def attention_fwd_fp8(q8, q_scale, k8, k_scale, v8t, v_scale, Nk: int, causal: bool = False,

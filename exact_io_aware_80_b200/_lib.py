@@ -11,7 +11,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libfa.so")
+# FA_LIBRARY selects another build of the same ABI, e.g. libfa_checks.so (device-side
+# index checks): a file name inside this package or an absolute path.
+LIB_PATH = os.path.join(_HERE, os.environ.get("FA_LIBRARY", "libfa.so"))
 
 FA_OK = 0
 FA_ERR_INVALID = -1
@@ -19,6 +21,7 @@ FA_ERR_UNSUPPORTED = -2
 FA_ERR_ALIGN = -3
 FA_ERR_CUDA = -4
 FA_ERR_TIMEOUT = -5
+FA_ERR_BOUNDS = -6
 FA_FP16 = 0
 FA_BF16 = 1
 
@@ -47,7 +50,10 @@ SIGNATURES = {
     "fa_fp8_quantize_qk": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "fa_fp8_v_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I]),
     "fa_fp8_quantize_v": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "fa_fp8_quantize_qkv": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "fa_fwd_merge": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_bwd_accumulate": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_lse_merge": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "fa_accumulate": (_I, [_P, _P, ctypes.c_longlong, _I, _I, _P]),
     "fa_cast_f32": (_I, [_P, _P, ctypes.c_longlong, _I, _P]),
@@ -172,10 +178,29 @@ def fa_fp8_quantize_v(v, v8t, scale, workspace, B, Hkv, Nk, d, dt, stream):
     return _check("fa_fp8_quantize_v", load().fa_fp8_quantize_v(v, v8t, scale, workspace, B, Hkv, Nk, d, dt, stream))
 
 
+def fa_fp8_quantize_qkv(q, k, v, q8, k8, v8t, q_scale, k_scale, v_scale, signs, workspace, B, Hq, Hkv, Nq, Nk, d, dt,
+                        stream):
+    return _check("fa_fp8_quantize_qkv", load().fa_fp8_quantize_qkv(q, k, v, q8, k8, v8t, q_scale, k_scale, v_scale,
+                                                                    signs, workspace, B, Hq, Hkv, Nq, Nk, d, dt,
+                                                                    stream))
+
+
 def fa_fwd_fp8(q8, q_scale, k8, k_scale, v8t, v_scale, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, rotated, dt,
                stream):
     return _check("fa_fwd_fp8", load().fa_fwd_fp8(q8, q_scale, k8, k_scale, v8t, v_scale, o, lse, B, Hq, Hkv, Nq, Nk,
                                                   d, int(causal), scale, int(rotated), dt, stream))
+
+
+def fa_fwd_merge(q, k, v, o, lse, acc_o, acc_lse, mode, B, Hq, Hkv, Nq, Nk, d, causal, scale, dt, stream):
+    return _check("fa_fwd_merge", load().fa_fwd_merge(q, k, v, o, lse, acc_o, acc_lse, mode, B, Hq, Hkv, Nq, Nk, d,
+                                                      int(causal), scale, dt, stream))
+
+
+def fa_bwd_accumulate(q, k, v, dout, lse, workspace, dq_acc, dk_acc, dv_acc, init, B, Hq, Hkv, Nq, Nk, d, causal,
+                      scale, dt, stream):
+    return _check("fa_bwd_accumulate", load().fa_bwd_accumulate(q, k, v, dout, lse, workspace, dq_acc, dk_acc, dv_acc,
+                                                                init, B, Hq, Hkv, Nq, Nk, d, int(causal), scale, dt,
+                                                                stream))
 
 
 def fa_lse_merge(o_acc, lse_acc, o_part, lse_part, o_out, B, N, H, d, mode, dt, stream):

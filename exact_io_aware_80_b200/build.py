@@ -1,11 +1,12 @@
 """Build libfa.so in-tree with nvcc for sm_100a.
 
-    python -m exact_io_aware_80_b200.build [--force] [--jobs N]
+    python -m exact_io_aware_80_b200.build [--force] [--jobs N] [--checks]
 
 Each .cu file under csrc/ is compiled to an object in csrc/_build/ (skipped
 when the object is newer than every source and header), then all objects are
-linked into exact_io_aware_80_b200/libfa.so.  No GPU is needed: nvcc
-cross-compiles.
+linked into exact_io_aware_80_b200/libfa.so.  --checks builds the same ABI with
+device-side index checks (FA_CHECKS) into csrc/_build_checks/ and
+libfa_checks.so.  No GPU is needed: nvcc cross-compiles.
 """
 from __future__ import annotations
 
@@ -20,7 +21,9 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(CSRC, "_build")
+BUILD_CHECKS = os.path.join(CSRC, "_build_checks")
 LIB = os.path.join(PKG, "libfa.so")
+LIB_CHECKS = os.path.join(PKG, "libfa_checks.so")
 ROOT = os.path.dirname(PKG)
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -41,8 +44,8 @@ def _newest_header() -> float:
     return max((os.path.getmtime(h) for h in hs), default=0.0)
 
 
-def _compile(src: str, force: bool, extra) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src: str, force: bool, extra, build_dir: str = BUILD) -> str:
+    obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
     if not force and os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(src), _newest_header()):
         return obj
     cmd = [nvcc()] + ARCH + FLAGS + list(extra) + os.environ.get("FA_NVCC_EXTRA", "").split() + ["-c", src, "-o", obj]
@@ -54,18 +57,24 @@ def _compile(src: str, force: bool, extra) -> str:
     return obj
 
 
-def build(force: bool = False, jobs: int = 0, extra=()) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, jobs: int = 0, extra=(), checks: bool = False) -> str:
+    """Build libfa.so, or with checks=True libfa_checks.so: the same sources compiled with
+    FA_CHECKS, whose kernels check their direct memory accesses against the tensors' sizes
+    and record FA_ERR_BOUNDS in the device status word instead of making the access."""
+    build_dir = BUILD_CHECKS if checks else BUILD
+    lib = LIB_CHECKS if checks else LIB
+    extra = list(extra) + (["-DFA_CHECKS"] if checks else [])
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     jobs = jobs or min(len(srcs), os.cpu_count() or 4)
     with cf.ThreadPoolExecutor(jobs) as ex:
-        objs = list(ex.map(lambda s: _compile(s, force, extra), srcs))
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        cmd = [nvcc()] + ARCH + ["-shared", "-o", LIB] + objs + ["-lcudart"]
+        objs = list(ex.map(lambda s: _compile(s, force, extra, build_dir), srcs))
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < max(os.path.getmtime(o) for o in objs):
+        cmd = [nvcc()] + ARCH + ["-shared", "-o", lib] + objs + ["-lcudart"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{' '.join(cmd)}\n{r.stdout}\n{r.stderr}")
-    return LIB
+    return lib
 
 
 def main():
@@ -73,9 +82,10 @@ def main():
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--jobs", type=int, default=0)
     ap.add_argument("--ptxas-verbose", action="store_true", help="print register / spill / smem usage")
+    ap.add_argument("--checks", action="store_true", help="build libfa_checks.so (device-side index checks)")
     a = ap.parse_args()
     extra = ["-Xptxas", "-v"] if a.ptxas_verbose else []
-    print(build(force=a.force or a.ptxas_verbose, jobs=a.jobs, extra=extra))
+    print(build(force=a.force or a.ptxas_verbose, jobs=a.jobs, extra=extra, checks=a.checks))
 
 
 if __name__ == "__main__":

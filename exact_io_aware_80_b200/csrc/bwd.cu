@@ -13,42 +13,66 @@ namespace {
 // ---------------------------------------------------------------------------
 // D = rowsum(dO * O)
 // ---------------------------------------------------------------------------
+// D / 8 threads share a row (16 bytes each), so a warp reads 256 contiguous bytes of
+// each of 32 / (D / 8) rows per load; each thread takes kRowsPerThread rows of one
+// (b, h), consecutive query positions, and issues all of their loads before any
+// arithmetic so that every thread has 2 * kRowsPerThread 16-byte loads in flight.
+// Rows are ordered (b, h, i) with i fastest, so the D values a warp writes are
+// contiguous.
+constexpr int kRowsPerThread = 4;
+
 template <typename T, int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs p) {
-  constexpr int TPR = D / 8;  // threads per row, 16 bytes each
-  const long R = (long)p.B * p.Nq * p.Hq;
-  const long gt = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long r = gt / TPR;
-  const int part = (int)(gt % TPR);
-  float acc = 0.f;
-  if (r < R) {
-    const uint4 o = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.o) + r * D) + part);
-    const uint4 g = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.dout) + r * D) + part);
-    const uint32_t ov[4] = {o.x, o.y, o.z, o.w};
-    const uint32_t gv[4] = {g.x, g.y, g.z, g.w};
+  constexpr int TPR = D / 8;         // threads per row
+  constexpr int RPW = 32 / TPR;      // rows per warp per load
+  constexpr int WROWS = RPW * kRowsPerThread;  // rows per warp
+  const int lane = threadIdx.x & 31;
+  const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int part = lane % TPR, sub = lane / TPR;
+  const long NqPad = (long)(p.Nq + WROWS - 1) / WROWS * WROWS;  // each warp stays inside one (b, h)
+  const long bh = warp * WROWS / NqPad;
+  if (bh >= (long)p.B * p.Hq) return;
+  const int i0 = (int)(warp * WROWS - bh * NqPad);
+  const long bb = bh / p.Hq;
+  const int h = (int)(bh % p.Hq);
+  uint4 o[kRowsPerThread], g[kRowsPerThread];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 a = Elem<T>::unpack(ov[i]), c = Elem<T>::unpack(gv[i]);
-      acc = fmaf(a.x, c.x, acc);
-      acc = fmaf(a.y, c.y, acc);
+  for (int k = 0; k < kRowsPerThread; ++k) {
+    const int i = i0 + k * RPW + sub;
+    const long off = ((bb * p.Nq + i) * p.Hq + h) * D;
+    if (i < p.Nq && FA_IN_BOUNDS(p.status, off + D - 1, (long)p.B * p.Nq * p.Hq * D)) {
+      o[k] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.o) + off) + part);
+      g[k] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.dout) + off) + part);
+    } else {
+      o[k] = g[k] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
 #pragma unroll
-  for (int w = 1; w < TPR; w <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
-  if (part == 0 && r < R) {
-    const long bb = r / ((long)p.Nq * p.Hq);
-    const int i = (int)((r / p.Hq) % p.Nq);
-    const int h = (int)(r % p.Hq);
-    p.dvec[(bb * p.Hq + h) * p.Nq + i] = acc;
+  for (int k = 0; k < kRowsPerThread; ++k) {
+    const uint32_t ov[4] = {o[k].x, o[k].y, o[k].z, o[k].w};
+    const uint32_t gv[4] = {g[k].x, g[k].y, g[k].z, g[k].w};
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 a = Elem<T>::unpack(ov[e]), c = Elem<T>::unpack(gv[e]);
+      acc = fmaf(a.x, c.x, acc);
+      acc = fmaf(a.y, c.y, acc);
+    }
+#pragma unroll
+    for (int w = 1; w < TPR; w <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
+    const int i = i0 + k * RPW + sub;
+    if (part == 0 && i < p.Nq && FA_IN_BOUNDS(p.status, bh * p.Nq + i, (long)p.B * p.Hq * p.Nq))
+      p.dvec[bh * p.Nq + i] = acc;
   }
 }
 
 template <typename T, int D>
 cudaError_t launch_pre_t(const BwdArgs& a, cudaStream_t s) {
-  const long R = (long)a.B * a.Nq * a.Hq;
-  const long threads = R * (D / 8);
-  const int blocks = (int)((threads + 255) / 256);
-  bwd_pre_kernel<T, D><<<blocks, 256, 0, s>>>(a);
+  constexpr int WROWS = (32 / (D / 8)) * kRowsPerThread;
+  const long warps = (long)a.B * a.Hq * ((a.Nq + WROWS - 1) / WROWS);
+  const long blocks = (warps + 7) / 8;
+  if (blocks > 0x7fffffffL) return cudaErrorInvalidValue;
+  bwd_pre_kernel<T, D><<<(unsigned)blocks, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 

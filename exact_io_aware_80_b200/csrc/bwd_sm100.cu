@@ -71,7 +71,42 @@ struct Params {
   float scale_log2;
   int* status;
   Dropout drop;  // DROP only
+  // ACC only: fp32 accumulators the results are added into (set when acc_init): acc0 = dK or dQ,
+  // acc1 = dV, laid out like the 16-bit outputs
+  float* acc0;
+  float* acc1;
+  int acc_init;
 };
+
+// One row of D fp32 TMEM columns, times `mul`, added into (or, with init, stored to) the fp32
+// row `dst` of an accumulator; the row is this thread's own, so no other thread touches it.
+// Every lane of the warp must call it (tcgen05.ld is warp-collective); lanes whose row lies
+// outside the tensor pass active = false and touch no memory.
+template <int D>
+__device__ __forceinline__ void acc_row(uint32_t taddr, float* dst, float mul, bool init, bool active) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int q = 0; q < D / 32; ++q) {
+    uint32_t x[32];
+    tmem_ld32(taddr + q * 32, x);
+    tmem_wait_ld();
+    reg_fence(x);
+    if (!active) continue;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float4 v = make_float4(__uint_as_float(x[4 * c]) * mul, __uint_as_float(x[4 * c + 1]) * mul,
+                             __uint_as_float(x[4 * c + 2]) * mul, __uint_as_float(x[4 * c + 3]) * mul);
+      if (!init) {
+        const float4 o = d4[q * 8 + c];
+        v.x += o.x;
+        v.y += o.y;
+        v.z += o.z;
+        v.w += o.w;
+      }
+      d4[q * 8 + c] = v;
+    }
+  }
+}
 
 // One row of D fp32 TMEM columns, times `mul`, as 16-bit values into a stage tile laid out as
 // a TMA box with 128-byte swizzle: 64-column panels of 128-byte rows, 16-byte chunk c of row r
@@ -171,7 +206,7 @@ struct DkdvSmem {
 // TMEM columns: S^T / P^T, dP^T / dS^T, dV, dK
 constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256, kColDK = 384;
 
-template <typename T, int D, bool CAUSAL, bool DROP>
+template <typename T, int D, bool CAUSAL, bool DROP, bool ACC = false>
 __global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -378,8 +413,9 @@ __global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
       const int h = hk * G + t / per_head;
       const int i = (mstart + t % per_head) * kT + tid;
       const long idx = ((long)b * p.Hq + h) * p.Nq + i;
-      lv = i < p.Nq ? -p.lse[idx] * kLog2e : -INFINITY;  // negated; rows past Nq get P = 0
-      dv = i < p.Nq ? -p.dvec[idx] : 0.f;                 // negated
+      const bool in = i < p.Nq && FA_IN_BOUNDS(p.status, idx, (long)p.B * p.Hq * p.Nq);
+      lv = in ? -p.lse[idx] * kLog2e : -INFINITY;  // negated; rows past Nq get P = 0
+      dv = in ? -p.dvec[idx] : 0.f;                 // negated
     };
     // LSE and D of query tile t sit in shared buffer t & 1; every elementwise thread
     // writes one entry and arrives on kBarLse + buffer.  Waiting for buffer t & 1
@@ -458,7 +494,14 @@ __global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
       }
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDone), 0, abort_flag, p.status));
-    if (ok) {
+    if (ACC && ok) {
+      // added into the fp32 accumulators, one key row per thread
+      tc_fence_after();
+      const long rowoff = (((long)b * p.Nk + key) * p.Hkv + hk) * D;
+      const bool active = key < p.Nk && FA_IN_BOUNDS(p.status, rowoff + D - 1, (long)p.B * p.Nk * p.Hkv * D);
+      acc_row<D>(tbase + lane_off + kColDV, p.acc1 + rowoff, DROP ? p.drop.inv_keep : 1.f, p.acc_init != 0, active);
+      acc_row<D>(tbase + lane_off + kColDK, p.acc0 + rowoff, p.scale, p.acc_init != 0, active);
+    } else if (ok) {
       // every MMA has run, so the Q and dO buffers are free: dV and dK leave through them by TMA
       // (rows past Nk are clipped by the tensor maps)
       tc_fence_after();
@@ -513,7 +556,7 @@ struct DqSmem {
 __host__ __device__ constexpr uint32_t col_s(int buf) { return 128u * buf; }
 constexpr uint32_t kColDP = 256, kColDQ = 384;
 
-template <typename T, int D, bool CAUSAL, bool DROP>
+template <typename T, int D, bool CAUSAL, bool DROP, bool ACC = false>
 __global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
     bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -693,8 +736,9 @@ __global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const float c = p.scale_log2;
     const long idx = ((long)b * p.Hq + h) * p.Nq + row;
-    const float nlse2 = row < p.Nq ? -p.lse[idx] * kLog2e : -INFINITY;  // rows past Nq get P = 0
-    const float ndrow = row < p.Nq ? -p.dvec[idx] : 0.f;
+    const bool in = row < p.Nq && FA_IN_BOUNDS(p.status, idx, (long)p.B * p.Hq * p.Nq);
+    const float nlse2 = in ? -p.lse[idx] * kLog2e : -INFINITY;  // rows past Nq get P = 0
+    const float ndrow = in ? -p.dvec[idx] : 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const uint32_t tS = tbase + lane_off + col_s(j & 1);
@@ -738,7 +782,12 @@ __global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
       mbar_arrive(bar(L::kBarDS));
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDone), 0, abort_flag, p.status));
-    if (ok) {
+    if (ACC && ok) {
+      tc_fence_after();
+      const long rowoff = (((long)b * p.Nq + row) * p.Hq + h) * D;
+      const bool active = row < p.Nq && FA_IN_BOUNDS(p.status, rowoff + D - 1, (long)p.B * p.Nq * p.Hq * D);
+      acc_row<D>(tbase + lane_off + kColDQ, p.acc0 + rowoff, p.scale, p.acc_init != 0, active);
+    } else if (ok) {
       // every MMA has run, so the Q buffer is free: dQ leaves through it by TMA (rows past Nq clipped)
       tc_fence_after();
       stage_row<T, D>(tbase + lane_off + kColDQ, sb + L::kOffQ, wq * 32 + lane, p.scale);
@@ -790,38 +839,46 @@ bool split_fits(K kern) {
   return fa.numRegs * kThreadsDrop >= 128 * (kRegsElem + kRegsCtrl + kRegsRng);
 }
 
-Params params(const BwdArgs& a, void* out0, void* out1) {
+Params params(const BwdArgs& a, void* out0, void* out1, float* acc0, float* acc1) {
   return Params{a.lse,  a.dvec,      out0,  out1, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, a.scale, a.scale * kLog2e, a.status,
-                Dropout{a.drop_thr, a.drop_inv_keep, a.seed_lo, a.seed_hi, a.drop_offset}};
+                Dropout{a.drop_thr, a.drop_inv_keep, a.seed_lo, a.seed_hi, a.drop_offset}, acc0, acc1, a.acc_init};
 }
 
 template <typename T, int D, bool CAUSAL>
 cudaError_t launch_dkdv(const BwdArgs& a, cudaStream_t s) {
   Maps m;
-  if (!make_maps(m, a, true, false)) return cudaErrorInvalidValue;
+  const bool acc = a.acc_k != nullptr;
+  if (!make_maps(m, a, !acc, false)) return cudaErrorInvalidValue;
   const bool drop = a.drop_p > 0.f;
-  auto kern = drop ? bwd_dkdv_sm100_kernel<T, D, CAUSAL, true> : bwd_dkdv_sm100_kernel<T, D, CAUSAL, false>;
+  if (acc && drop) return cudaErrorInvalidValue;
+  auto kern = acc ? bwd_dkdv_sm100_kernel<T, D, CAUSAL, false, true>
+                  : drop ? bwd_dkdv_sm100_kernel<T, D, CAUSAL, true> : bwd_dkdv_sm100_kernel<T, D, CAUSAL, false>;
   const int smem = DkdvSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   if (drop && !split_fits(kern)) return cudaErrorInvalidConfiguration;
   dim3 grid(a.Hkv, (a.Nk + kT - 1) / kT, a.B);
-  kern<<<grid, drop ? kThreadsDrop : kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, m.dk, m.dv, params(a, a.dk, a.dv));
+  kern<<<grid, drop ? kThreadsDrop : kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, m.dk, m.dv,
+                                                          params(a, a.dk, a.dv, a.acc_k, a.acc_v));
   return cudaGetLastError();
 }
 
 template <typename T, int D, bool CAUSAL>
 cudaError_t launch_dq(const BwdArgs& a, cudaStream_t s) {
   Maps m;
-  if (!make_maps(m, a, false, true)) return cudaErrorInvalidValue;
+  const bool acc = a.acc_q != nullptr;
+  if (!make_maps(m, a, false, !acc)) return cudaErrorInvalidValue;
   const bool drop = a.drop_p > 0.f;
-  auto kern = drop ? bwd_dq_sm100_kernel<T, D, CAUSAL, true> : bwd_dq_sm100_kernel<T, D, CAUSAL, false>;
+  if (acc && drop) return cudaErrorInvalidValue;
+  auto kern = acc ? bwd_dq_sm100_kernel<T, D, CAUSAL, false, true>
+                  : drop ? bwd_dq_sm100_kernel<T, D, CAUSAL, true> : bwd_dq_sm100_kernel<T, D, CAUSAL, false>;
   const int smem = drop ? DqSmem<D, true>::kBytes : DqSmem<D, false>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   if (drop && !split_fits(kern)) return cudaErrorInvalidConfiguration;
   dim3 grid(a.Hq, (a.Nq + kT - 1) / kT, a.B);
-  kern<<<grid, drop ? kThreadsDrop : kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, m.dq, params(a, a.dq, nullptr));
+  kern<<<grid, drop ? kThreadsDrop : kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, m.dq,
+                                                          params(a, a.dq, nullptr, a.acc_q, nullptr));
   return cudaGetLastError();
 }
 

@@ -21,6 +21,21 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 // Device status word codes (mirrors fa_status in fa.h).
 constexpr int kStatusTimeout = -5;
+constexpr int kStatusBounds = -6;
+
+// Index checks of the FA_CHECKS build (libfa_checks.so): FA_IN_BOUNDS(status, i, n) is true
+// when 0 <= i < n; otherwise it records kStatusBounds in the status word (no trap) and the
+// caller skips the access.  In the normal build it is the constant true and costs nothing.
+__device__ __forceinline__ bool in_bounds_or_flag(int* status, long long i, long long n) {
+  if (i >= 0 && i < n) return true;
+  if (status) atomicCAS(status, 0, kStatusBounds);
+  return false;
+}
+#ifdef FA_CHECKS
+#define FA_IN_BOUNDS(status, i, n) ::fa::in_bounds_or_flag((status), (long long)(i), (long long)(n))
+#else
+#define FA_IN_BOUNDS(status, i, n) ((void)(status), (void)(i), (void)(n), true)
+#endif
 
 // Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, "Parallel random
 // numbers: as easy as 1, 2, 3", SC 2011): per round, with M0 = 0xD2511F53 and

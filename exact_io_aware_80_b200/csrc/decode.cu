@@ -44,9 +44,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(DecodeArgs p)
   const int hi = min(lo + p.chunk, n);
   const long part0 = ((long)b * p.Hq + (long)hk * G) * S + s;  // (b, h = hk*G + g, s) = part0 + g*S
 
+  const long nparts = (long)p.B * p.Hq * S;
   if (hi <= lo) {
-    for (int i = tid; i < G * D; i += kThreads) p.o_part[(part0 + (long)(i / D) * S) * D + (i % D)] = 0.f;
-    if (tid < G) p.lse_part[part0 + (long)tid * S] = -INFINITY;
+    for (int i = tid; i < G * D; i += kThreads) {
+      const long oi = (part0 + (long)(i / D) * S) * D + (i % D);
+      if (FA_IN_BOUNDS(p.status, oi, nparts * D)) p.o_part[oi] = 0.f;
+    }
+    if (tid < G && FA_IN_BOUNDS(p.status, part0 + (long)tid * S, nparts)) p.lse_part[part0 + (long)tid * S] = -INFINITY;
     return;
   }
   const int ntiles = (hi - lo + kTileN - 1) / kTileN;
@@ -181,8 +185,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(DecodeArgs p)
       L += red_l[w * kRows + g] * f;
       O += red_o[(w * kRows + g) * D + col] * f;
     }
-    p.o_part[(part0 + (long)g * S) * D + col] = O / L;
-    if (col == 0) p.lse_part[part0 + (long)g * S] = (M + lg2(L)) * kLn2;
+    const long oi = (part0 + (long)g * S) * D + col;
+    if (FA_IN_BOUNDS(p.status, oi, nparts * D)) p.o_part[oi] = O / L;
+    if (col == 0 && FA_IN_BOUNDS(p.status, part0 + (long)g * S, nparts)) p.lse_part[part0 + (long)g * S] = (M + lg2(L)) * kLn2;
   }
 }
 
@@ -192,6 +197,7 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(CombineArgs p) {
   const int h = blockIdx.x, b = blockIdx.y, col = threadIdx.x;
   const int S = p.num_splits;
   const long base = ((long)b * p.Hq + h) * S;
+  if (!FA_IN_BOUNDS(p.status, base + S - 1, (long)p.B * p.Hq * S)) return;
   float M = -INFINITY;
   for (int s = 0; s < S; ++s) M = fmaxf(M, p.lse_part[base + s]);
   float L = 0.f, O = 0.f;
@@ -206,8 +212,9 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(CombineArgs p) {
   uint16_t* go = static_cast<uint16_t*>(p.o) + ((long)b * p.Hq + h) * D;
   T v;
   if constexpr (Elem<T>::kBf16) v = __float2bfloat16_rn(out); else v = __float2half_rn(out);
-  go[col] = *reinterpret_cast<uint16_t*>(&v);
-  if (col == 0) p.lse[(long)b * p.Hq + h] = L > 0.f ? M + logf(L) : -INFINITY;
+  if (FA_IN_BOUNDS(p.status, ((long)b * p.Hq + h) * D + col, (long)p.B * p.Hq * D)) go[col] = *reinterpret_cast<uint16_t*>(&v);
+  if (col == 0 && FA_IN_BOUNDS(p.status, (long)b * p.Hq + h, (long)p.B * p.Hq))
+    p.lse[(long)b * p.Hq + h] = L > 0.f ? M + logf(L) : -INFINITY;
 }
 
 template <typename T, int D>

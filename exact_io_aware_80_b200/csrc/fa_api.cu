@@ -93,6 +93,7 @@ const char* fa_status_string(fa_status s) {
     case FA_ERR_ALIGN: return "pointer not aligned";
     case FA_ERR_CUDA: return "CUDA error";
     case FA_ERR_TIMEOUT: return "kernel wait timed out";
+    case FA_ERR_BOUNDS: return "device-side index check failed";
   }
   return "unknown status";
 }
@@ -116,7 +117,7 @@ fa_status fa_fp8_quantize_qk(const void* x, void* x8, float* scales, const float
   fa_status st = check_shape(B, H, H, N, N, d, 0, dt);
   if (st != FA_OK) return st;
   if (!aligned16(x) || !aligned16(x8) || !aligned4(scales) || (signs && !aligned4(signs))) return FA_ERR_ALIGN;
-  fa::Fp8QuantArgs a{x, x8, scales, signs, nullptr, B, H, N, d, dt == FA_BF16 ? 1 : 0};
+  fa::Fp8QuantArgs a{x, x8, scales, signs, nullptr, B, H, N, d, dt == FA_BF16 ? 1 : 0, status_ptr()};
   return from_cuda(fa::launch_fp8_quant_qk(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -131,8 +132,24 @@ fa_status fa_fp8_quantize_v(const void* v, void* v8t, float* scale, void* worksp
   fa_status st = check_shape(B, Hkv, Hkv, Nk, Nk, d, 0, dt);
   if (st != FA_OK) return st;
   if (!aligned16(v) || !aligned16(v8t) || !aligned16(workspace) || !aligned4(scale)) return FA_ERR_ALIGN;
-  fa::Fp8QuantArgs a{v, v8t, scale, nullptr, static_cast<float*>(workspace), B, Hkv, Nk, d, dt == FA_BF16 ? 1 : 0};
+  fa::Fp8QuantArgs a{v, v8t, scale, nullptr, static_cast<float*>(workspace), B, Hkv, Nk, d, dt == FA_BF16 ? 1 : 0,
+                     status_ptr()};
   return from_cuda(fa::launch_fp8_quant_v(a, static_cast<cudaStream_t>(stream)));
+}
+
+fa_status fa_fp8_quantize_qkv(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8t,
+                              float* q_scale, float* k_scale, float* v_scale, const float* signs, void* workspace,
+                              int B, int Hq, int Hkv, int Nq, int Nk, int d, fa_dtype dt, fa_stream_t stream) {
+  if (!q || !k || !v || !q8 || !k8 || !v8t || !q_scale || !k_scale || !v_scale || !workspace) return FA_ERR_INVALID;
+  fa_status st = check_shape(B, Hq, Hkv, Nq, Nk, d, 0, dt);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q8) || !aligned16(k8) || !aligned16(v8t) ||
+      !aligned16(workspace) || !aligned4(q_scale) || !aligned4(k_scale) || !aligned4(v_scale) ||
+      (signs && !aligned4(signs)))
+    return FA_ERR_ALIGN;
+  fa::Fp8QkvArgs a{q, k, v, q8, k8, v8t, q_scale, k_scale, v_scale, signs, static_cast<float*>(workspace),
+                   B, Hq, Hkv, Nq, Nk, d, dt == FA_BF16 ? 1 : 0, status_ptr()};
+  return from_cuda(fa::launch_fp8_quant_qkv(a, static_cast<cudaStream_t>(stream)));
 }
 
 fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const float* k_scale, const void* v8t,
@@ -177,6 +194,25 @@ fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse)) return FA_ERR_ALIGN;
   fa::AttnArgs a{q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal ? 1 : 0, scale, dt == FA_BF16 ? 1 : 0, status_ptr(),
                  block_mask};
+  if (!a.status) return FA_ERR_CUDA;
+  if (!fa::fwd_sm100_supported(a)) return FA_ERR_CUDA;
+  return from_cuda(fa::launch_fwd_sm100(a, static_cast<cudaStream_t>(stream)));
+}
+
+fa_status fa_fwd_merge(const void* q, const void* k, const void* v, void* o, float* lse, float* acc_o,
+                       float* acc_lse, int mode, int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                       float scale, fa_dtype dt, fa_stream_t stream) {
+  if (!q || !k || !v || !o || !lse || !acc_o || !acc_lse) return FA_ERR_INVALID;
+  if (mode < 0 || mode > 2) return FA_ERR_INVALID;
+  fa_status st = check_shape(B, Hq, Hkv, Nq, Nk, d, causal, dt);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(acc_o) || !aligned4(lse) ||
+      !aligned4(acc_lse))
+    return FA_ERR_ALIGN;
+  fa::AttnArgs a{q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal ? 1 : 0, scale, dt == FA_BF16 ? 1 : 0, status_ptr()};
+  a.acc_o = acc_o;
+  a.acc_lse = acc_lse;
+  a.acc_mode = mode;
   if (!a.status) return FA_ERR_CUDA;
   if (!fa::fwd_sm100_supported(a)) return FA_ERR_CUDA;
   return from_cuda(fa::launch_fwd_sm100(a, static_cast<cudaStream_t>(stream)));
@@ -366,7 +402,7 @@ fa_status fa_decode_combine(const void* workspace, void* o, float* lse, const in
   if (!aligned16(workspace) || !aligned16(o) || !aligned4(lse) || !aligned4(seqlens_k)) return FA_ERR_ALIGN;
   const float* o_part = static_cast<const float*>(workspace);
   const float* lse_part = o_part + (size_t)B * Hq * num_splits * d;
-  fa::CombineArgs a{o_part, lse_part, seqlens_k, o, lse, B, Hq, d, num_splits, dt == FA_BF16 ? 1 : 0};
+  fa::CombineArgs a{o_part, lse_part, seqlens_k, o, lse, B, Hq, d, num_splits, dt == FA_BF16 ? 1 : 0, status_ptr()};
   return from_cuda(fa::launch_decode_combine(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -392,3 +428,32 @@ fa_status fa_get_device_status(fa_stream_t stream) {
 }
 
 }  // extern "C"
+
+fa_status fa_bwd_accumulate(const void* q, const void* k, const void* v, const void* dout, const float* lse,
+                            const void* workspace, float* dq_acc, float* dk_acc, float* dv_acc, int init, int B,
+                            int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale, fa_dtype dt,
+                            fa_stream_t stream) {
+  if (!q || !k || !v || !dout || !lse || !workspace || !dq_acc || !dk_acc || !dv_acc) return FA_ERR_INVALID;
+  if (init < 0 || init > 3) return FA_ERR_INVALID;
+  fa_status st = check_shape(B, Hq, Hkv, Nq, Nk, d, causal, dt);
+  if (st != FA_OK) return st;
+  const void* p16[] = {q, k, v, dout, workspace, dq_acc, dk_acc, dv_acc};
+  for (const void* p : p16)
+    if (!aligned16(p)) return FA_ERR_ALIGN;
+  if (!aligned4(lse)) return FA_ERR_ALIGN;
+  if (!fa::tma_available()) return FA_ERR_CUDA;
+  fa::BwdArgs a{q, k, v, nullptr, dout, lse, nullptr, nullptr, nullptr, static_cast<float*>(const_cast<void*>(workspace)),
+                B, Hq, Hkv, Nq, Nk, d, causal ? 1 : 0, scale, dt == FA_BF16 ? 1 : 0, status_ptr()};
+  if (!a.status) return FA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  fa::BwdArgs kv = a;
+  kv.acc_k = dk_acc;
+  kv.acc_v = dv_acc;
+  kv.acc_init = (init & 2) ? 1 : 0;
+  cudaError_t e = fa::launch_bwd_dkdv_sm100(kv, s);
+  if (e != cudaSuccess) return from_cuda(e);
+  fa::BwdArgs qa = a;
+  qa.acc_q = dq_acc;
+  qa.acc_init = (init & 1) ? 1 : 0;
+  return from_cuda(fa::launch_bwd_dq_sm100(qa, s));
+}

@@ -14,11 +14,22 @@
 //   * V: one scale per (batch, kv head) over all keys, codes stored transposed
 //     as [B, Hkv, d, Nk_pad] (Nk_pad = Nk rounded up to 16; zero codes in the
 //     padding) so that the P V product reads V K-major.
-// These kernels move Nq x d (or Nk x d) 16-bit values once; they are bound by
-// HBM bandwidth and run once per input, outside the attention kernel.
+//
+// These kernels move each 16-bit input once (V twice: its per-head scale
+// needs the amax of every key first) and are bound by HBM bandwidth.  One CTA
+// of 128 threads takes one 128-row block of one head: the block is staged in
+// shared memory with coalesced 16-byte cp.async copies (a row is contiguous,
+// rows of one head are H * d elements apart), each thread then works on one
+// row in registers (rotation, block amax, division, E4M3 packing), and the
+// codes leave through shared memory with coalesced 16-byte stores.  The Q, K
+// and V-amax blocks of a forward pass run in one persistent launch whose CTAs
+// stage their next block while working on the current one; V's transposing
+// encode is a second launch, since it needs the head's amax.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -32,21 +43,6 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
-}
-
-template <typename T>
-__device__ __forceinline__ void load_row(const T* src, float* y, int d) {
-  const uint4* s4 = reinterpret_cast<const uint4*>(src);
-  for (int i = 0; i < d / 8; ++i) {
-    const uint4 w = s4[i];
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 f = Elem<T>::unpack(u[k]);
-      y[8 * i + 2 * k] = f.x;
-      y[8 * i + 2 * k + 1] = f.y;
-    }
-  }
 }
 
 // In-place unnormalised Walsh-Hadamard transform of y[0..D), fp32 butterflies
@@ -77,23 +73,64 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 
 __device__ __forceinline__ float scale_of(float amax) { return amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f; }
 
-// grid (row blocks, H, B), 128 threads: thread r quantises row 128 blockIdx.x + r.
+// Staged rows: D 16-bit values plus 16 bytes of padding, so that 8 threads reading
+// 16 bytes of 8 consecutive rows hit distinct banks (row stride = 4 banks mod 32).
+template <int D>
+struct Stage {
+  static constexpr int kRowBytes = 2 * D + 16;
+  static constexpr int kBytes = kRows * kRowBytes;
+  static constexpr int kChunks = D / 8;  // 16-byte chunks per row
+};
+
+// Rows n0 .. n0 + 127 of head h, batch b of x [B, N, H, D] into the stage (rows
+// past N as zeros): 16-byte cp.async copies, consecutive threads on consecutive
+// chunks.  Issued only; the caller commits and waits.
 template <typename T, int D>
-__global__ void __launch_bounds__(kRows) quant_qk_kernel(const T* __restrict__ x, uint8_t* __restrict__ x8,
-                                                          float* __restrict__ scales, const float* __restrict__ signs,
-                                                          int N, int H) {
-  __shared__ float red[4];
-  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int n = j * kRows + threadIdx.x;
-  const bool valid = n < N;
-  const long row = ((long)b * N + n) * H + h;
-  float y[D];
-  if (valid) {
-    load_row(x + row * D, y, D);
-  } else {
-#pragma unroll
-    for (int i = 0; i < D; ++i) y[i] = 0.f;
+__device__ __forceinline__ void issue_rows(const T* x, uint8_t* st, int N, int H, int b, int h, int n0) {
+  using S = Stage<D>;
+  const uint32_t base = smem_u32(st);
+#pragma unroll 4
+  for (int e = threadIdx.x; e < kRows * S::kChunks; e += kRows) {
+    const int r = e / S::kChunks, c = e % S::kChunks;
+    const int n = n0 + r;
+    const bool ok = n < N;
+    const T* src = x + (((long)b * N + (ok ? n : 0)) * H + h) * D + 8 * c;
+    cp_async16(base + r * S::kRowBytes + 16 * c, src, ok);
   }
+}
+template <typename T, int D>
+__device__ __forceinline__ void stage_rows(const T* x, uint8_t* st, int N, int H, int b, int h, int n0) {
+  issue_rows<T, D>(x, st, N, H, b, h, n0);
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+}
+
+// Row r of the stage as fp32.
+template <typename T, int D>
+__device__ __forceinline__ void read_row(const uint8_t* st, int r, float (&y)[D]) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(st + r * Stage<D>::kRowBytes);
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) {
+    const uint4 w = s4[i];
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = Elem<T>::unpack(u[k]);
+      y[8 * i + 2 * k] = f.x;
+      y[8 * i + 2 * k + 1] = f.y;
+    }
+  }
+}
+
+// One 128-row block of Q or K: (signs, Walsh-Hadamard), block amax, scale, E4M3 codes.
+template <typename T, int D>
+__device__ __forceinline__ void quant_rows_block(const QuantJob& job, const float* signs, int j, int h, int b, int B,
+                                                 uint8_t* st, float* red, int* status) {
+  using S = Stage<D>;
+  const int r = threadIdx.x;
+  float y[D];
+  read_row<T, D>(st, r, y);
   if (signs) {
 #pragma unroll
     for (int i = 0; i < D; ++i) y[i] = y[i] * signs[i];  // exact: +-1
@@ -102,11 +139,12 @@ __global__ void __launch_bounds__(kRows) quant_qk_kernel(const T* __restrict__ x
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < D; ++i) amax = fmaxf(amax, fabsf(y[i]));
-  amax = block_max(amax, red);
+  amax = block_max(amax, red);  // its barriers also order every read of the stage before the writes below
   const float s = scale_of(amax);
-  if (threadIdx.x == 0) scales[((long)b * H + h) * gridDim.x + j] = s;
-  if (!valid) return;
-  uint4* dst = reinterpret_cast<uint4*>(x8 + row * D);
+  if (r == 0 && FA_IN_BOUNDS(status, ((long)b * job.H + h) * job.nblk + j, (long)B * job.H * job.nblk))
+    job.scales[((long)b * job.H + h) * job.nblk + j] = s;
+  // codes of row r over the first D bytes of its own stage row
+  uint4* row = reinterpret_cast<uint4*>(st + r * S::kRowBytes);
 #pragma unroll
   for (int i = 0; i < D / 16; ++i) {
     uint32_t w[4];
@@ -117,98 +155,220 @@ __global__ void __launch_bounds__(kRows) quant_qk_kernel(const T* __restrict__ x
       const uint32_t hi = e4m3x2(__fdiv_rn(y[c + 2], s), __fdiv_rn(y[c + 3], s));
       w[k] = lo | (hi << 16);
     }
-    dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    row[i] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  __syncthreads();
+  // D code bytes per row, 16 at a time, consecutive threads on consecutive chunks of a row
+  constexpr int C8 = D / 16;
+  const int n0 = j * kRows;
+#pragma unroll 4
+  for (int e = threadIdx.x; e < kRows * C8; e += kRows) {
+    const int rr = e / C8, c = e % C8;
+    const int n = n0 + rr;
+    const long ci = (((long)b * job.N + n) * job.H + h) * D + 16 * c;
+    if (n < job.N && FA_IN_BOUNDS(status, ci + 15, (long)B * job.N * job.H * D))
+      *reinterpret_cast<uint4*>(job.x8 + ci) = *reinterpret_cast<const uint4*>(st + rr * S::kRowBytes + 16 * c);
   }
 }
 
-// grid (row blocks, Hkv, B): amax of every 128-key block of V into part[b][h][j].
+// Amax of one staged 128-key block of V into part[b][h][j] (rows past N were staged as zeros).
 template <typename T, int D>
-__global__ void __launch_bounds__(kRows) v_amax_kernel(const T* __restrict__ v, float* __restrict__ part, int Nk,
-                                                        int H) {
-  __shared__ float red[4];
-  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int n = j * kRows + threadIdx.x;
+__device__ __forceinline__ void v_amax_block(const QuantJob& job, int j, int h, int b, int B, const uint8_t* st,
+                                             float* red, int* status) {
+  float y[D];
+  read_row<T, D>(st, threadIdx.x, y);
   float amax = 0.f;
-  if (n < Nk) {
-    float y[D];
-    load_row(v + (((long)b * Nk + n) * H + h) * D, y, D);
 #pragma unroll
-    for (int i = 0; i < D; ++i) amax = fmaxf(amax, fabsf(y[i]));
-  }
+  for (int i = 0; i < D; ++i) amax = fmaxf(amax, fabsf(y[i]));
   amax = block_max(amax, red);
-  if (threadIdx.x == 0) part[((long)b * H + h) * gridDim.x + j] = amax;
+  if (threadIdx.x == 0 && FA_IN_BOUNDS(status, ((long)b * job.H + h) * job.nblk + j, (long)B * job.H * job.nblk))
+    job.scales[((long)b * job.H + h) * job.nblk + j] = amax;
 }
 
-// grid (row blocks, Hkv, B): quantise 128 keys of V with the head's scale and
-// write them transposed, [d][128 keys] per block, through shared memory.
+// One persistent launch over up to three jobs (Q rows, K rows, V block maxima).  The flat
+// block index walks job 0's blocks (j fastest, then h, then b), then job 1's, then job 2's;
+// CTA i takes blocks i, i + G, i + 2G, ... and stages block i + G into its second buffer
+// while it works on block i, so the copies overlap the arithmetic.
+struct BlockRef {
+  int job, j, h, b;
+};
+__device__ __forceinline__ BlockRef block_ref(const QuantJobs& jobs, long id, int B) {
+  int k = 0;
+  while (k < jobs.n - 1 && id >= (long)jobs.job[k].nblk * jobs.job[k].H * B) {
+    id -= (long)jobs.job[k].nblk * jobs.job[k].H * B;
+    ++k;
+  }
+  const int nb = jobs.job[k].nblk, H = jobs.job[k].H;
+  return BlockRef{k, (int)(id % nb), (int)((id / nb) % H), (int)(id / ((long)nb * H))};
+}
+
+template <typename T, int D>
+__device__ __forceinline__ void issue_block(const QuantJobs& jobs, const BlockRef& r, uint8_t* st) {
+  const QuantJob& job = jobs.job[r.job];
+  issue_rows<T, D>(static_cast<const T*>(job.x), st, job.N, job.H, r.b, r.h, r.j * kRows);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kRows) quant_kernel(QuantJobs jobs, const float* __restrict__ signs, int B,
+                                                      long total) {
+  extern __shared__ __align__(16) uint8_t q_smem[];  // two stages
+  __shared__ float red[4];
+  uint8_t* stage[2] = {q_smem, q_smem + Stage<D>::kBytes};
+  long id = blockIdx.x;
+  if (id < total) issue_block<T, D>(jobs, block_ref(jobs, id, B), stage[0]);
+  cp_async_commit();
+  for (int it = 0; id < total; ++it, id += gridDim.x) {
+    const long nxt = id + gridDim.x;
+    if (nxt < total) issue_block<T, D>(jobs, block_ref(jobs, nxt, B), stage[(it + 1) & 1]);
+    cp_async_commit();
+    cp_async_wait<1>();  // this block's copies have landed (the next block's may still fly)
+    __syncthreads();
+    const BlockRef r = block_ref(jobs, id, B);
+    const QuantJob& job = jobs.job[r.job];
+    if (job.kind == kQuantRows)
+      quant_rows_block<T, D>(job, signs, r.j, r.h, r.b, B, stage[it & 1], red, jobs.status);
+    else
+      v_amax_block<T, D>(job, r.j, r.h, r.b, B, stage[it & 1], red, jobs.status);
+    __syncthreads();  // every thread is done with this buffer before it is refilled
+  }
+  cp_async_wait<0>();
+}
+
+// One 128-key block of V: the head's scale from the block maxima, then codes written
+// transposed ([d][128 keys] for the block) through shared memory.
 template <typename T, int D>
 __global__ void __launch_bounds__(kRows) v_quant_kernel(const T* __restrict__ v, const float* __restrict__ part,
                                                          uint8_t* __restrict__ v8t, float* __restrict__ scale,
-                                                         int Nk, int H, int Npad) {
-  __shared__ __align__(16) uint8_t tile[D][kRows + 16];
+                                                         int Nk, int H, int Npad, int* status) {
+  using S = Stage<D>;
+  constexpr int kOutRow = kRows + 16;  // bytes per transposed code row (+ padding)
+  extern __shared__ __align__(16) uint8_t vq_smem[];  // the stage, then D transposed code rows
+  uint8_t* st = vq_smem;
+  uint8_t* out = vq_smem + S::kBytes;
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int nb = gridDim.x;
+  stage_rows<T, D>(v, st, Nk, H, b, h, j * kRows);
   float amax = 0.f;
   const float* ph = part + ((long)b * H + h) * nb;
   for (int i = 0; i < nb; ++i) amax = fmaxf(amax, ph[i]);
   const float s = scale_of(amax);
-  if (j == 0 && threadIdx.x == 0) scale[(long)b * H + h] = s;
-  const int r = threadIdx.x, n = j * kRows + r;
-  if (n < Nk) {
-    float y[D];
-    load_row(v + (((long)b * Nk + n) * H + h) * D, y, D);
+  if (j == 0 && threadIdx.x == 0 && FA_IN_BOUNDS(status, (long)b * H + h, (long)gridDim.z * H)) scale[(long)b * H + h] = s;
+  // thread c < D encodes column c of the block: keys 0..127 (rows past Nk were staged as zeros)
+  for (int c = threadIdx.x; c < D; c += kRows) {
+#pragma unroll 2
+    for (int k16 = 0; k16 < kRows / 16; ++k16) {
+      uint32_t w[4];
 #pragma unroll
-    for (int c = 0; c < D; c += 2) {
-      const uint16_t p = e4m3x2(__fdiv_rn(y[c], s), __fdiv_rn(y[c + 1], s));
-      tile[c][r] = (uint8_t)(p & 0xFF);
-      tile[c + 1][r] = (uint8_t)(p >> 8);
+      for (int q = 0; q < 4; ++q) {
+        float f[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = 16 * k16 + 4 * q + e;
+          const uint16_t raw = *reinterpret_cast<const uint16_t*>(st + key * S::kRowBytes + 2 * c);
+          f[e] = Elem<T>::unpack((uint32_t)raw).x;
+        }
+        w[q] = (uint32_t)e4m3x2(__fdiv_rn(f[0], s), __fdiv_rn(f[1], s)) |
+               ((uint32_t)e4m3x2(__fdiv_rn(f[2], s), __fdiv_rn(f[3], s)) << 16);
+      }
+      *reinterpret_cast<uint4*>(out + c * kOutRow + 16 * k16) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-  } else {
-#pragma unroll
-    for (int c = 0; c < D; ++c) tile[c][r] = 0;
   }
   __syncthreads();
-  // row c of the block: keys 128 j .. 128 j + 127, clipped to Npad (a multiple of 16)
+  // row c of the block: keys 128 j .. 128 j + 127, clipped to Npad (a multiple of 16); codes of
+  // keys past Nk are zeros
   const int nkeys = min(kRows, Npad - j * kRows);
   uint8_t* base = v8t + ((long)b * H + h) * D * (long)Npad + (long)j * kRows;
   for (int e = threadIdx.x; e < D * (kRows / 16); e += kRows) {
     const int c = e / (kRows / 16), q = e % (kRows / 16);
-    if (16 * q < nkeys) {
-      const uint32_t* t4 = reinterpret_cast<const uint32_t*>(&tile[c][16 * q]);
-      *reinterpret_cast<uint4*>(base + (long)c * Npad + 16 * q) = make_uint4(t4[0], t4[1], t4[2], t4[3]);
-    }
+    const long vi = (((long)b * H + h) * D + c) * (long)Npad + (long)j * kRows + 16 * q;
+    if (16 * q < nkeys && FA_IN_BOUNDS(status, vi + 15, (long)gridDim.z * H * D * Npad))
+      *reinterpret_cast<uint4*>(base + (long)c * Npad + 16 * q) = *reinterpret_cast<const uint4*>(out + c * kOutRow + 16 * q);
   }
 }
 
+template <int D>
+struct VQuantSmem {
+  static constexpr int kBytes = Stage<D>::kBytes + D * (kRows + 16);
+};
+
 template <typename T, int D>
-cudaError_t launch_qk(const Fp8QuantArgs& a, cudaStream_t s) {
-  dim3 grid((a.N + kRows - 1) / kRows, a.H, a.B);
-  quant_qk_kernel<T, D><<<grid, kRows, 0, s>>>(static_cast<const T*>(a.x), static_cast<uint8_t*>(a.x8), a.scales,
-                                              a.signs, a.N, a.H);
+cudaError_t launch_jobs(const QuantJobs& jobs, const float* signs, int B, cudaStream_t s) {
+  long blocks = 0;
+  for (int k = 0; k < jobs.n; ++k) blocks += (long)jobs.job[k].nblk * jobs.job[k].H * B;
+  if (blocks < 1 || blocks > 0x7fffffffL) return cudaErrorInvalidValue;
+  constexpr int smem = 2 * Stage<D>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(quant_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_kernel<T, D>, kRows, smem);
+  if (e != cudaSuccess) return e;
+  const long grid = std::min<long>(blocks, (long)std::max(per_sm, 1) * device_sm_count());
+  quant_kernel<T, D><<<(unsigned)grid, kRows, smem, s>>>(jobs, signs, B, blocks);
   return cudaGetLastError();
 }
 
 template <typename T, int D>
-cudaError_t launch_v(const Fp8QuantArgs& a, cudaStream_t s) {
-  dim3 grid((a.N + kRows - 1) / kRows, a.H, a.B);
-  v_amax_kernel<T, D><<<grid, kRows, 0, s>>>(static_cast<const T*>(a.x), a.work, a.N, a.H);
-  cudaError_t e = cudaGetLastError();
+cudaError_t launch_v_quant(const void* v, const float* part, void* v8t, float* scale, int B, int H, int Nk,
+                           int* status, cudaStream_t s) {
+  dim3 grid((Nk + kRows - 1) / kRows, H, B);
+  constexpr int smem = VQuantSmem<D>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(v_quant_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  v_quant_kernel<T, D><<<grid, kRows, 0, s>>>(static_cast<const T*>(a.x), a.work, static_cast<uint8_t*>(a.x8),
-                                             a.scales, a.N, a.H, (a.N + 15) / 16 * 16);
+  v_quant_kernel<T, D><<<grid, kRows, smem, s>>>(static_cast<const T*>(v), part, static_cast<uint8_t*>(v8t), scale, Nk,
+                                                H, (Nk + 15) / 16 * 16, status);
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t jobs_d(const QuantJobs& jobs, const float* signs, int B, bool bf16, cudaStream_t s) {
+  return bf16 ? launch_jobs<__nv_bfloat16, D>(jobs, signs, B, s) : launch_jobs<__half, D>(jobs, signs, B, s);
+}
+template <int D>
+cudaError_t vq_d(const void* v, const float* part, void* v8t, float* scale, int B, int H, int Nk, bool bf16,
+                 int* status, cudaStream_t s) {
+  return bf16 ? launch_v_quant<__nv_bfloat16, D>(v, part, v8t, scale, B, H, Nk, status, s)
+              : launch_v_quant<__half, D>(v, part, v8t, scale, B, H, Nk, status, s);
+}
+
+QuantJob rows_job(const void* x, void* x8, float* scales, int H, int N) {
+  return QuantJob{x, static_cast<uint8_t*>(x8), scales, N, H, (N + kRows - 1) / kRows, kQuantRows};
+}
+QuantJob amax_job(const void* v, float* part, int H, int N) {
+  return QuantJob{v, nullptr, part, N, H, (N + kRows - 1) / kRows, kQuantAmax};
 }
 
 }  // namespace
 
 cudaError_t launch_fp8_quant_qk(const Fp8QuantArgs& a, cudaStream_t s) {
-  if (a.bf16) return a.d == 128 ? launch_qk<__nv_bfloat16, 128>(a, s) : launch_qk<__nv_bfloat16, 64>(a, s);
-  return a.d == 128 ? launch_qk<__half, 128>(a, s) : launch_qk<__half, 64>(a, s);
+  QuantJobs jobs{};
+  jobs.n = 1;
+  jobs.status = a.status;
+  jobs.job[0] = rows_job(a.x, a.x8, a.scales, a.H, a.N);
+  return a.d == 128 ? jobs_d<128>(jobs, a.signs, a.B, a.bf16, s) : jobs_d<64>(jobs, a.signs, a.B, a.bf16, s);
 }
 
 cudaError_t launch_fp8_quant_v(const Fp8QuantArgs& a, cudaStream_t s) {
-  if (a.bf16) return a.d == 128 ? launch_v<__nv_bfloat16, 128>(a, s) : launch_v<__nv_bfloat16, 64>(a, s);
-  return a.d == 128 ? launch_v<__half, 128>(a, s) : launch_v<__half, 64>(a, s);
+  QuantJobs jobs{};
+  jobs.n = 1;
+  jobs.status = a.status;
+  jobs.job[0] = amax_job(a.x, a.work, a.H, a.N);
+  cudaError_t e = a.d == 128 ? jobs_d<128>(jobs, nullptr, a.B, a.bf16, s) : jobs_d<64>(jobs, nullptr, a.B, a.bf16, s);
+  if (e != cudaSuccess) return e;
+  return a.d == 128 ? vq_d<128>(a.x, a.work, a.x8, a.scales, a.B, a.H, a.N, a.bf16, a.status, s)
+                    : vq_d<64>(a.x, a.work, a.x8, a.scales, a.B, a.H, a.N, a.bf16, a.status, s);
+}
+
+cudaError_t launch_fp8_quant_qkv(const Fp8QkvArgs& a, cudaStream_t s) {
+  QuantJobs jobs{};
+  jobs.n = 3;
+  jobs.status = a.status;
+  jobs.job[0] = rows_job(a.q, a.q8, a.q_scale, a.Hq, a.Nq);
+  jobs.job[1] = rows_job(a.k, a.k8, a.k_scale, a.Hkv, a.Nk);
+  jobs.job[2] = amax_job(a.v, a.work, a.Hkv, a.Nk);
+  cudaError_t e = a.d == 128 ? jobs_d<128>(jobs, a.signs, a.B, a.bf16, s) : jobs_d<64>(jobs, a.signs, a.B, a.bf16, s);
+  if (e != cudaSuccess) return e;
+  return a.d == 128 ? vq_d<128>(a.v, a.work, a.v8t, a.v_scale, a.B, a.Hkv, a.Nk, a.bf16, a.status, s)
+                    : vq_d<64>(a.v, a.work, a.v8t, a.v_scale, a.B, a.Hkv, a.Nk, a.bf16, a.status, s);
 }
 
 }  // namespace fa

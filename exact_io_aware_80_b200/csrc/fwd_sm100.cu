@@ -121,7 +121,54 @@ struct Params {
   int nqb, nkb;  // 128-row blocks of Nq and Nk (FP8 scales and the block-sparse table)
   const uint8_t* block_mask;  // block-sparse only: [B, Hq, nqb, nkb], nonzero = computed
   Dropout drop;               // dropout only
+  // fp32 accumulator of the merged result (ACC only): O [B,Nq,Hq,D], LSE [B,Hq,Nq]; acc_mode 0: set,
+  // 1: merge and keep, 2: merge into the outputs o, lse
+  float* acc_o;
+  float* acc_lse;
+  int acc_mode;
 };
+
+// Log-sum-exp merge of this launch's row (O_part = r * inv, LSE_part = lse) with the fp32
+// accumulator row ("FlashAttention 심층 분석", Flash-Decoding: partial results over disjoint key
+// ranges combine by their log-sum-exp).  Mode 0 stores the part; otherwise the merged row
+// replaces r (inv becomes 1) and lse, and mode 1 also stores it back.
+template <int D>
+__device__ __forceinline__ void merge_acc_row(const Params& p, long orow, long lrow, uint32_t (&r)[D], float& inv,
+                                              float& lse) {
+  float4* acc = reinterpret_cast<float4*>(p.acc_o + orow * D);
+  if (p.acc_mode == 0) {
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c)
+      acc[c] = make_float4(__uint_as_float(r[4 * c]) * inv, __uint_as_float(r[4 * c + 1]) * inv,
+                           __uint_as_float(r[4 * c + 2]) * inv, __uint_as_float(r[4 * c + 3]) * inv);
+    p.acc_lse[lrow] = lse;
+    return;
+  }
+  const float la = p.acc_lse[lrow];
+  const float mx = fmaxf(la, lse);
+  float wa = 0.f, wp = 0.f;
+  if (mx != -INFINITY) {
+    wa = ex2((la - mx) * kLog2e);
+    wp = ex2((lse - mx) * kLog2e);
+  }
+  const float s = wa + wp;
+  const float ia = s > 0.f ? wa / s : 0.f, ip = s > 0.f ? wp * inv / s : 0.f;
+#pragma unroll
+  for (int c = 0; c < D / 4; ++c) {
+    const float4 a = acc[c];
+    const float4 m = make_float4(ia * a.x + ip * __uint_as_float(r[4 * c]), ia * a.y + ip * __uint_as_float(r[4 * c + 1]),
+                                 ia * a.z + ip * __uint_as_float(r[4 * c + 2]),
+                                 ia * a.w + ip * __uint_as_float(r[4 * c + 3]));
+    r[4 * c] = __float_as_uint(m.x);
+    r[4 * c + 1] = __float_as_uint(m.y);
+    r[4 * c + 2] = __float_as_uint(m.z);
+    r[4 * c + 3] = __float_as_uint(m.w);
+    if (p.acc_mode == 1) acc[c] = m;
+  }
+  lse = s > 0.f ? mx + lg2(s) * kLn2 : -INFINITY;
+  if (p.acc_mode == 1) p.acc_lse[lrow] = lse;
+  inv = 1.f;
+}
 
 // Work tile w of the persistent schedule: row block, query head, batch.  Causal
 // row blocks are enumerated longest first (all heads and batches of one length
@@ -146,7 +193,7 @@ __device__ __forceinline__ Work work_at(const Params& p, int w) {
   return x;
 }
 
-template <typename T, int D, bool CAUSAL, bool F8, bool SPARSE, bool DROP>
+template <typename T, int D, bool CAUSAL, bool F8, bool SPARSE, bool DROP, bool ACC = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, Params p) {
@@ -169,7 +216,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // K/V tile >= j below nblk that either query tile marks (j itself for dense attention)
   auto mask_row = [&](const Work& x, int t) -> const uint8_t* {
     const int qb = kTiles * x.mblk + t;
-    return qb < p.nqb ? p.block_mask + (((long)x.b * p.Hq + x.hq) * p.nqb + qb) * p.nkb : nullptr;
+    if (qb >= p.nqb) return nullptr;
+    const long mi = (((long)x.b * p.Hq + x.hq) * p.nqb + qb) * p.nkb;
+    if (!FA_IN_BOUNDS(p.status, mi + p.nkb - 1, (long)p.B * p.Hq * p.nqb * p.nkb)) return nullptr;
+    return p.block_mask + mi;
   };
   auto next_vis = [&](const Work& x, int j, int nblk) {
     if constexpr (SPARSE) {
@@ -415,11 +465,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j0 >= nblk) {
           // block-sparse work tile with no K/V tile: every row attends to nothing
           if (row < p.Nq) {
-            uint4* orow =
-                reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + (((long)b * p.Nq + row) * p.Hq + h) * D);
+            const long oi = (((long)b * p.Nq + row) * p.Hq + h) * D;
+            if (FA_IN_BOUNDS(p.status, oi + D - 1, (long)p.B * p.Nq * p.Hq * D)) {
+              uint4* orow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + oi);
 #pragma unroll
-            for (int i = 0; i < D / 8; ++i) orow[i] = make_uint4(0u, 0u, 0u, 0u);
-            p.lse[((long)b * p.Hq + h) * p.Nq + row] = -INFINITY;
+              for (int i = 0; i < D / 8; ++i) orow[i] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            const long li = ((long)b * p.Hq + h) * p.Nq + row;
+            if (FA_IN_BOUNDS(p.status, li, (long)p.B * p.Hq * p.Nq)) p.lse[li] = -INFINITY;
           }
           continue;
         }
@@ -430,7 +483,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (SPARSE) mrow = mask_row(x, t);
       const int hk = h / (p.Hq / p.Hkv);
       float cq = c;  // FP8: times the Q tile's block scale
-      if constexpr (F8) cq = c * p.q_scale[((long)b * p.Hq + h) * p.nqb + min(row_first / kBM, p.nqb - 1)];
+      if constexpr (F8) {
+        const long si = ((long)b * p.Hq + h) * p.nqb + min(row_first / kBM, p.nqb - 1);
+        cq = FA_IN_BOUNDS(p.status, si, (long)p.B * p.Hq * p.nqb) ? c * p.q_scale[si] : 0.f;
+      }
       float m_ref = -INFINITY, l = 0.f;
       for (int j = j0; j < nblk; j = next_vis(x, j + 1, nblk), ++g) {
         uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit c = (this row, key j kBN + c) kept
@@ -481,7 +537,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         float cj = cq;  // FP8: times the K block's scale
-        if constexpr (F8) cj = cq * p.k_scale[((long)b * p.Hkv + hk) * p.nkb + j];
+        if constexpr (F8) {
+          const long si = ((long)b * p.Hkv + hk) * p.nkb + j;
+          cj = FA_IN_BOUNDS(p.status, si, (long)p.B * p.Hkv * p.nkb) ? cq * p.k_scale[si] : 0.f;
+        }
         const int kbase = j * kBN;
         bool on = true;  // block-sparse: this query tile computes block (., j)
         if constexpr (SPARSE) on = mrow && mrow[j];
@@ -578,12 +637,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         // O / l as 16-bit into the stage buffer, laid out as the TMA box expects: 64-column
         // panels of 128-byte rows, 16-byte chunk c of row r at chunk c ^ (r & 7)
         float num = 1.f;  // FP8: V's scale; dropout: 1 / (1 - p)
-        if constexpr (F8) num = p.v_scale[(long)b * p.Hkv + hk];
+        if constexpr (F8) num = FA_IN_BOUNDS(p.status, (long)b * p.Hkv + hk, (long)p.B * p.Hkv) ? p.v_scale[(long)b * p.Hkv + hk] : 0.f;
         if constexpr (DROP) num = p.drop.inv_keep;
         // block-sparse: a row that saw no visible key keeps m_ref = -inf (its l holds only the
         // clamped polynomial exp2 of -inf): O = 0 and LSE = -inf
         const bool any = SPARSE ? (l > 0.f && m_ref != -INFINITY) : l > 0.f;
-        const float inv = any ? num / l : 0.f;
+        float inv = any ? num / l : 0.f;
+        float lse_row = any ? (m_ref + lg2(l)) * kLn2 : -INFINITY;
+        if constexpr (ACC) {
+          const long orow = ((long)b * p.Nq + row) * p.Hq + h, lrow = ((long)b * p.Hq + h) * p.Nq + row;
+          if (row < p.Nq && FA_IN_BOUNDS(p.status, orow, (long)p.B * p.Nq * p.Hq) &&
+              FA_IN_BOUNDS(p.status, lrow, (long)p.B * p.Hq * p.Nq))
+            merge_acc_row<D>(p, orow, lrow, r, inv, lse_row);
+        }
         const int rr = wq * 32 + lane;
         const uint32_t srow = sb + L::kOffStage + rr * 128;
         auto o2 = [&](int i) { return Elem<T>::pack(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv); };
@@ -593,7 +659,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                        o2(8 * c + 4), o2(8 * c + 6));
         fence_proxy_async_smem();
         mbar_arrive(bar(L::kBarStageFull + t));
-        if (row < p.Nq) p.lse[((long)b * p.Hq + h) * p.Nq + row] = any ? (m_ref + lg2(l)) * kLn2 : -INFINITY;
+        if (row < p.Nq && FA_IN_BOUNDS(p.status, ((long)b * p.Hq + h) * p.Nq + row, (long)p.B * p.Hq * p.Nq))
+          p.lse[((long)b * p.Hq + h) * p.Nq + row] = lse_row;
         if (wq == 0 && lane == 0) {
           // one thread of the tile stores it; rows past Nq are clipped by the tensor map
           ok = mbar_wait(bar(L::kBarStageFull + t), we & 1, abort_flag, p.status);
@@ -638,7 +705,16 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   if (num_work > (1ll << 31) - 1) return cudaErrorInvalidValue;
   Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, a.scale * kLog2e, a.status, num_mblk, (int)num_work,
            nullptr, nullptr, nullptr, (a.Nq + kBM - 1) / kBM, (a.Nk + kBN - 1) / kBN, a.block_mask,
-           Dropout{a.drop_thr, a.drop_inv_keep, a.seed_lo, a.seed_hi, a.drop_offset}};
+           Dropout{a.drop_thr, a.drop_inv_keep, a.seed_lo, a.seed_hi, a.drop_offset}, a.acc_o, a.acc_lse, a.acc_mode};
+  if (a.acc_o) {
+    auto kern = fwd_sm100_kernel<T, D, CAUSAL, false, false, false, true>;
+    const int smem = Smem<D, false>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)std::min<long long>(num_work, device_sm_count());
+    kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mo, p);
+    return cudaGetLastError();
+  }
   if (a.drop_p > 0.f) {
     auto kern = fwd_sm100_kernel<T, D, CAUSAL, false, false, true>;
     const int smem = Smem<D, false>::kBytes;
@@ -689,7 +765,8 @@ cudaError_t launch_f8(const Fp8AttnArgs& a, cudaStream_t s) {
   if (num_work > (1ll << 31) - 1) return cudaErrorInvalidValue;
   const float sl2 = a.scale * kLog2e / (a.rotated ? (float)D : 1.f);
   Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, sl2, a.status, num_mblk, (int)num_work,
-           a.q_scale, a.k_scale, a.v_scale, (a.Nq + kBM - 1) / kBM, (a.Nk + kBN - 1) / kBN, nullptr, Dropout{}};
+           a.q_scale, a.k_scale, a.v_scale, (a.Nq + kBM - 1) / kBM, (a.Nk + kBN - 1) / kBN, nullptr, Dropout{},
+           nullptr, nullptr, 0};
   auto kern = fwd_sm100_kernel<T, D, CAUSAL, true, false, false>;
   const int smem = Smem<D, true>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -25,6 +25,11 @@ struct AttnArgs {
   uint32_t drop_thr = 0;
   float drop_inv_keep = 1.f;
   uint32_t seed_lo = 0, seed_hi = 0, drop_offset = 0;
+  // merge into an fp32 accumulator (acc_o != nullptr): O [B,Nq,Hq,d] and LSE [B,Hq,Nq] fp32;
+  // acc_mode 0: acc = this result; 1: acc = merge(acc, result); 2: o, lse = merge(acc, result)
+  float* acc_o = nullptr;
+  float* acc_lse = nullptr;
+  int acc_mode = 0;
 };
 
 struct BwdArgs {
@@ -47,6 +52,12 @@ struct BwdArgs {
   uint32_t drop_thr = 0;
   float drop_inv_keep = 1.f;
   uint32_t seed_lo = 0, seed_hi = 0, drop_offset = 0;
+  // add into fp32 accumulators instead of writing 16-bit gradients (acc_q / acc_k / acc_v !=
+  // nullptr): dQ [B,Nq,Hq,d], dK and dV [B,Nk,Hkv,d]; acc_init: set instead of add
+  float* acc_q = nullptr;
+  float* acc_k = nullptr;
+  float* acc_v = nullptr;
+  int acc_init = 0;
 };
 
 struct DecodeArgs {
@@ -71,6 +82,7 @@ struct CombineArgs {
   float* lse;
   int B, Hq, d, num_splits;
   int bf16;
+  int* status = nullptr;  // index checks of the FA_CHECKS build
 };
 
 // FP8 operand preparation (fp8_quant.cu).  Q/K: x [B,N,H,d] 16-bit -> x8 codes [B,N,H,d],
@@ -85,6 +97,34 @@ struct Fp8QuantArgs {
   float* work;
   int B, H, N, d;
   int bf16;
+  int* status = nullptr;  // index checks of the FA_CHECKS build
+};
+
+// One quantization job of the fused launch: E4M3 codes and block scales of the rows of
+// x [B, N, H, d] (kQuantRows), or the amax of every 128-row block of x into `scales`
+// (kQuantAmax, the first pass over V).
+constexpr int kQuantRows = 0, kQuantAmax = 1;
+struct QuantJob {
+  const void* x;
+  uint8_t* x8;
+  float* scales;
+  int N, H, nblk, kind;
+};
+struct QuantJobs {
+  QuantJob job[3];
+  int n;
+  int* status;  // index checks of the FA_CHECKS build
+};
+// Q, K and V of one forward pass quantized together (two launches).
+struct Fp8QkvArgs {
+  const void *q, *k, *v;
+  void *q8, *k8, *v8t;
+  float *q_scale, *k_scale, *v_scale;
+  const float* signs;
+  float* work;
+  int B, Hq, Hkv, Nq, Nk, d;
+  int bf16;
+  int* status = nullptr;  // index checks of the FA_CHECKS build
 };
 
 // FP8 forward: E4M3 Q/K codes [B,N,H,d] with block scales, V codes transposed
@@ -144,6 +184,7 @@ bool fwd_sm100_supported(const AttnArgs& a);
 cudaError_t launch_fwd_fp8_sm100(const Fp8AttnArgs& a, cudaStream_t s);
 cudaError_t launch_fp8_quant_qk(const Fp8QuantArgs& a, cudaStream_t s);
 cudaError_t launch_fp8_quant_v(const Fp8QuantArgs& a, cudaStream_t s);
+cudaError_t launch_fp8_quant_qkv(const Fp8QkvArgs& a, cudaStream_t s);
 
 cudaError_t launch_bwd_preprocess(const BwdArgs& a, cudaStream_t s);
 // Backward dK/dV and dQ on tcgen05 / TMEM / TMA, d = 128 and 64.

@@ -6,21 +6,22 @@ r ("contiguous"), or 2W parts with rank r owning parts r and 2W - 1 - r
 queries, keys and values of its parts, concatenated in that order.  In step
 s = 0 .. W-1 rank r holds the keys and values of rank c = (r - s) mod W and
 attends each of its query parts a to each held key part b (causal: b < a all
-keys, b == a the causal diagonal, b > a nothing) with the 16-bit forward
-kernel, folding each partial (O, LSE) into that query part's fp32 accumulator
-with the log-sum-exp merge kernel; meanwhile it sends the keys and values it
-holds to rank r + 1 and receives the next from rank r - 1 (point-to-point sends
-over the process group, NCCL between GPUs).  After W steps every rank holds
+keys, b == a the causal diagonal, b > a nothing) with the forward kernel, whose
+epilogue folds the chunk's result into that query part's fp32 accumulator by
+log-sum-exp (fa_fwd_merge: no 16-bit rounding of partial results); meanwhile
+it sends the keys and values it holds to rank r + 1 and receives the next from
+rank r - 1 (point-to-point sends over the process group, NCCL between GPUs).  After W steps every rank holds
 exact attention of its queries over the whole sequence ("FlashAttention 심층
 분석", "Flash-Decoding": attention over disjoint key ranges merges exactly by
 log-sum-exp; the koritips note names ring attention for context lengths past
 one GPU).
 
 Backward: with the rows' LSE (from the forward) and D = rowsum(dO * O), each
-(query part, key part) pair contributes exact partial gradients (the dQ and
-dK/dV kernels on that pair); dQ partials are summed in fp32 on the query's
-rank, and the fp32 dK/dV sums of the held key parts travel around the ring
-with their keys and values and reach their owner after one last hop.
+(query part, key part) pair contributes exact partial gradients, which the dQ
+and dK/dV kernels add straight into fp32 accumulators (fa_bwd_accumulate);
+dQ sums stay on the query's rank, and the fp32 dK/dV sums of the held key
+parts travel around the ring with their keys and values and reach their owner
+after one last hop.  Only the final results are rounded to 16 bits.
 
 `ring_schedule` is the pure schedule; `ring_attention_fwd` / `ring_attention_bwd`
 run it over a process group with the library's kernels (or, for host-side
@@ -72,35 +73,24 @@ def ring_schedule(rank: int, world: int, causal: bool, layout: str = "contiguous
 
 
 class _CudaOps:
-    """The library's kernels: partial attention (fa_fwd) and the log-sum-exp merge (fa_lse_merge)."""
+    """The library's kernels: the forward with its fp32 log-sum-exp merge (fa_fwd_merge), the
+    backward preprocess, the backward adding into fp32 accumulators (fa_bwd_accumulate) and the
+    final casts."""
 
     def __init__(self, torch, scale):
         self.torch, self.scale = torch, scale
 
-    def partial(self, q, k, v, causal):
+    def attend(self, q, k, v, causal, o_acc, lse_acc, out, lse_out, mode):
+        """Attention of q over one key chunk, merged into (o_acc, lse_acc) by log-sum-exp.
+
+        mode 0: the accumulator takes this chunk's result; 1: merge and keep; 2: merge into
+        out, lse_out (the last chunk).  out, lse_out are written in every mode."""
         torch = self.torch
         B, N, Hq, d = q.shape
         _, Nk, Hkv, _ = k.shape
-        o = torch.empty_like(q)
-        lse = torch.empty(B, Hq, N, device=q.device, dtype=torch.float32)
-        _lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, Nk, d,
-                    causal, self.scale, _dtype(torch, q), torch.cuda.current_stream(q.device).cuda_stream)
-        return o, lse
-
-    def merge(self, acc, part, last):
-        torch = self.torch
-        o_acc, lse_acc, out, first = acc
-        o_p, lse_p = part
-        B, N, H, d = o_p.shape
-        mode = 0 if first else (2 if last else 1)
-        if mode == 0 and last:  # a single chunk: its partial is the answer
-            out.copy_(o_p)
-            lse_acc.copy_(lse_p)
-            return
-        _lib.fa_lse_merge(o_acc.data_ptr(), lse_acc.data_ptr(), o_p.data_ptr(), lse_p.data_ptr(),
-                          out.data_ptr() if mode == 2 else 0, B, N, H, d, mode, _dtype(torch, o_p),
-                          torch.cuda.current_stream(o_p.device).cuda_stream)
-
+        _lib.fa_fwd_merge(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_out.data_ptr(),
+                          o_acc.data_ptr(), lse_acc.data_ptr(), mode, B, Hq, Hkv, N, Nk, d, causal, self.scale,
+                          _dtype(torch, q), torch.cuda.current_stream(q.device).cuda_stream)
 
     # ----------------------------------------------------------------- backward
     def preprocess(self, q, k, v, o, do, lse):
@@ -113,32 +103,20 @@ class _CudaOps:
                                _dtype(torch, q), torch.cuda.current_stream(q.device).cuda_stream)
         return ws
 
-    def partial_bwd(self, q, k, v, o, do, lse, ws, causal):
-        """dQ, dK, dV contributions (16-bit) of one chunk pair, with the rows' LSE and D."""
+    def accumulate_bwd(self, q, k, v, do, lse, ws, causal, dq_acc, dk_acc, dv_acc, init_q, init_kv):
+        """The dQ, dK, dV contributions of one chunk pair added into fp32 accumulators (or set, per init flag)."""
         torch = self.torch
         B, N, Hq, d = q.shape
         _, Nk, Hkv, _ = k.shape
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(), dq.data_ptr(),
-                dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), B, Hq, Hkv, N, Nk, d, causal, self.scale,
-                _dtype(torch, q), torch.cuda.current_stream(q.device).cuda_stream)
-        _lib.fa_bwd_dkdv(*args)
-        _lib.fa_bwd_dq(*args)
-        return dq, dk, dv
-
-    def accumulate(self, acc, part, init):
-        torch = self.torch
-        _lib.fa_accumulate(acc.data_ptr(), part.data_ptr(), part.numel(), init, _dtype(torch, part),
-                           torch.cuda.current_stream(part.device).cuda_stream)
+        _lib.fa_bwd_accumulate(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), lse.data_ptr(), ws.data_ptr(),
+                               dq_acc.data_ptr(), dk_acc.data_ptr(), dv_acc.data_ptr(),
+                               (1 if init_q else 0) | (2 if init_kv else 0), B, Hq, Hkv, N, Nk, d, causal,
+                               self.scale, _dtype(torch, q), torch.cuda.current_stream(q.device).cuda_stream)
 
     def cast(self, acc, out):
         torch = self.torch
         _lib.fa_cast_f32(acc.data_ptr(), out.data_ptr(), out.numel(), _dtype(torch, out),
                          torch.cuda.current_stream(out.device).cuda_stream)
-
-
-def _dtype(torch, t):
-    return _lib.FA_BF16 if t.dtype == torch.bfloat16 else _lib.FA_FP16
 
 
 def _dtype(torch, t):
@@ -157,7 +135,7 @@ def _split_lse(t, P):
 
 
 def _fwd_rank(torch, ops, sched, q_parts, held_kv):
-    """Forward of one rank: partials of every scheduled (query part, key part) pair merged per query part.
+    """Forward of one rank: every scheduled (query part, key part) pair attended and merged per query part.
 
     held_kv(step) -> list of (k, v) parts held at that step.  Returns lists of O and LSE per own part.
     """
@@ -170,13 +148,15 @@ def _fwd_rank(torch, ops, sched, q_parts, held_kv):
     outs = [torch.empty_like(qp) for qp in q_parts]
     lses = [torch.empty(B, Hq, n, device=qp.device, dtype=torch.float32) for qp in q_parts]
     accs = [torch.empty(B, n, Hq, d, device=qp.device, dtype=torch.float32) for qp in q_parts]
+    acc_lses = [torch.empty(B, Hq, n, device=qp.device, dtype=torch.float32) for qp in q_parts]
     first = [True] * P
     for s, _, pairs in sched:
         kv = held_kv(s)
         for ia, ib, mode in pairs:
-            part = ops.partial(q_parts[ia], kv[ib][0], kv[ib][1], mode == "causal")
             remaining[ia] -= 1
-            ops.merge((accs[ia], lses[ia], outs[ia], first[ia]), part, remaining[ia] == 0)
+            m = 0 if first[ia] else (2 if remaining[ia] == 0 else 1)
+            ops.attend(q_parts[ia], kv[ib][0], kv[ib][1], mode == "causal", accs[ia], acc_lses[ia], outs[ia],
+                       lses[ia], m)
             first[ia] = False
     for ia in range(P):
         if first[ia]:  # no key part attends to these queries (cannot happen for these schedules)
@@ -231,7 +211,7 @@ def ring_attention_fwd(q, k, v, causal: bool = False, scale: float | None = None
                        layout: str = "contiguous"):
     """Ring attention over a process group; q, k, v are this rank's parts concatenated ([B, n, H, d]).
 
-    Returns this rank's O [B, n, Hq, d] and LSE [B, Hq, n].  `ops` (partial, merge) defaults to the
+    Returns this rank's O [B, n, Hq, d] and LSE [B, Hq, n].  `ops` (attend) defaults to the
     library's CUDA kernels; the sends and receives of the keys and values overlap each step's compute.
     """
     import torch
@@ -263,8 +243,9 @@ def ring_attention_fwd(q, k, v, causal: bool = False, scale: float | None = None
     return torch.cat(outs, dim=1), torch.cat(lses, dim=2)
 
 
-def _bwd_rank(torch, ops, sched, qp, op, dop, lp, held, add_kv_grad):
-    """Backward of one rank: dQ sums per own part; per held key part, add_kv_grad(step, ib, dk, dv)."""
+def _bwd_rank(torch, ops, sched, qp, op, dop, lp, held, kv_acc):
+    """Backward of one rank: dQ sums per own part; the dK/dV contributions of held part ib at step s are
+    added into kv_acc(s, ib) -> (dk_acc, dv_acc, init)."""
     P = len(qp)
     wss = [ops.preprocess(qp[i], qp[i], qp[i], op[i], dop[i], lp[i]) for i in range(P)]
     B, n, Hq, d = qp[0].shape
@@ -273,11 +254,10 @@ def _bwd_rank(torch, ops, sched, qp, op, dop, lp, held, add_kv_grad):
     for s, _, pairs in sched:
         kv = held(s)
         for ia, ib, mode in pairs:
-            dq_p, dk_p, dv_p = ops.partial_bwd(qp[ia], kv[ib][0], kv[ib][1], op[ia], dop[ia], lp[ia], wss[ia],
-                                               mode == "causal")
-            ops.accumulate(dq_acc[ia], dq_p, first[ia])
+            dk_acc, dv_acc, init_kv = kv_acc(s, ib)
+            ops.accumulate_bwd(qp[ia], kv[ib][0], kv[ib][1], dop[ia], lp[ia], wss[ia], mode == "causal",
+                               dq_acc[ia], dk_acc, dv_acc, first[ia], init_kv)
             first[ia] = False
-            add_kv_grad(s, ib, dk_p, dv_p)
     dq = [torch.empty_like(x) for x in qp]
     for i in range(P):
         if first[i]:
@@ -315,14 +295,14 @@ def ring_attention_bwd_local(q, k, v, o, do, lse, world: int, causal: bool = Fal
         def held(s, sched=sched):
             return [(kg[b], vg[b]) for b in owned_parts(sched[s][1], world, layout)]
 
-        def add(s, ib, dk_p, dv_p, sched=sched):
+        def kv_acc(s, ib, sched=sched):
             b = owned_parts(sched[s][1], world, layout)[ib]
-            ops.accumulate(dk_acc[b], dk_p, kv_first[b])
-            ops.accumulate(dv_acc[b], dv_p, kv_first[b])
+            init = kv_first[b]
             kv_first[b] = False
+            return dk_acc[b], dv_acc[b], init
 
         dqs = _bwd_rank(torch, ops, sched, [qg[a] for a in mine], [og[a] for a in mine], [dog[a] for a in mine],
-                        [lg[a] for a in mine], held, add)
+                        [lg[a] for a in mine], held, kv_acc)
         for ia, a in enumerate(mine):
             dq[:, a * n:(a + 1) * n] = dqs[ia]
     dk, dv = torch.empty_like(k), torch.empty_like(v)
@@ -376,12 +356,9 @@ def ring_attention_bwd(q, k, v, o, do, lse, causal: bool = False, scale: float |
         if s + 1 < world:  # the keys and values of the next step travel while this step computes
             pending = _p2p(dist, group, nxt, prv, [t for x in cur_kv for t in x], [t for x in kv[(s + 1) % 2] for t in x])
         for ia, ib, mode in pairs:
-            dq_p, dk_p, dv_p = ops.partial_bwd(qp[ia], cur_kv[ib][0], cur_kv[ib][1], op[ia], dop[ia], lp[ia],
-                                               wss[ia], mode == "causal")
-            ops.accumulate(dq_acc[ia], dq_p, first[ia])
+            ops.accumulate_bwd(qp[ia], cur_kv[ib][0], cur_kv[ib][1], dop[ia], lp[ia], wss[ia], mode == "causal",
+                               dq_acc[ia], acc[s % 2][ib][0], acc[s % 2][ib][1], first[ia], False)
             first[ia] = False
-            ops.accumulate(acc[s % 2][ib][0], dk_p, False)
-            ops.accumulate(acc[s % 2][ib][1], dv_p, False)
         if s + 1 < world:
             # the held parts' gradient sums move on with them, after this step's contributions
             for r_ in _p2p(dist, group, nxt, prv, [t for x in acc[s % 2] for t in x],

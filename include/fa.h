@@ -53,7 +53,8 @@ typedef enum {
   FA_ERR_UNSUPPORTED = -2, /* d not in {64, 128}, unknown dtype, size beyond a stated limit */
   FA_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned */
   FA_ERR_CUDA = -4,        /* a CUDA runtime/driver call or a launch failed */
-  FA_ERR_TIMEOUT = -5      /* a kernel's bounded wait ran out (device status word) */
+  FA_ERR_TIMEOUT = -5,     /* a kernel's bounded wait ran out (device status word) */
+  FA_ERR_BOUNDS = -6       /* a device-side index check failed (libfa_checks.so only; device status word) */
 } fa_status;
 
 typedef enum { FA_FP16 = 0, FA_BF16 = 1 } fa_dtype;
@@ -262,6 +263,21 @@ fa_status fa_fp8_quantize_v(const void* v, void* v8t, float* scale, void* worksp
                             int d, fa_dtype dt, fa_stream_t stream);
 
 /*
+ * Q, K and V of one FP8 forward pass quantized together, in two launches (the
+ * Q and K rows with the V block maxima, then V's transposing encode): the same
+ * codes and scales as fa_fp8_quantize_qk on q and on k (both with `signs`)
+ * and fa_fp8_quantize_v on v.  q [B, Nq, Hq, d], k and v [B, Nk, Hkv, d]
+ * 16-bit; q8 [B, Nq, Hq, d] and k8 [B, Nk, Hkv, d] bytes with q_scale
+ * [B, Hq, ceil(Nq / 128)] and k_scale [B, Hkv, ceil(Nk / 128)]; v8t
+ * [B, Hkv, d, Nk_pad] bytes with v_scale [B, Hkv]; workspace as sized by
+ * fa_fp8_v_workspace_bytes(B, Hkv, Nk).  Tensors and workspace 16-byte
+ * aligned, scales and signs 4-byte aligned.
+ */
+fa_status fa_fp8_quantize_qkv(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8t,
+                              float* q_scale, float* k_scale, float* v_scale, const float* signs, void* workspace,
+                              int B, int Hq, int Hkv, int Nq, int Nk, int d, fa_dtype dt, fa_stream_t stream);
+
+/*
  * FP8 forward.  q8 [B, Nq, Hq, 128] and k8 [B, Nk, Hkv, 128] E4M3 codes with
  * scales [B, Hq, ceil(Nq / 128)] and [B, Hkv, ceil(Nk / 128)]; v8t [B, Hkv,
  * 128, Nk_pad] with scale [B, Hkv] (as written by the quantizers above).
@@ -289,6 +305,40 @@ fa_status fa_lse_merge(float* o_acc, float* lse_acc, const void* o_part, const f
                        int N, int H, int d, int mode, fa_dtype dt, fa_stream_t stream);
 
 /*
+ * Forward over one key/value chunk merged into an fp32 accumulator by
+ * log-sum-exp ("FlashAttention 심층 분석", "Flash-Decoding": attention over
+ * disjoint key ranges combines exactly by the ranges' log-sum-exp) -- the
+ * fa_fwd kernel with the merge done in its epilogue, so the partial result is
+ * never rounded to 16 bits.  acc_o fp32 [B, Nq, Hq, d] and acc_lse fp32
+ * [B, Hq, Nq] are the caller's accumulator.  mode 0: acc = this chunk's result;
+ * 1: acc = merge(acc, result); 2: o and lse = merge(acc, result), acc left as
+ * it was (the last chunk).  o [B, Nq, Hq, d] (dt) and lse are written in every
+ * mode (modes 0 and 1: the running result).  A row with no visible key in
+ * either gets O = 0 and LSE = -inf.  Otherwise as fa_fwd; acc_o 16-byte
+ * aligned, acc_lse 4-byte aligned.
+ */
+fa_status fa_fwd_merge(const void* q, const void* k, const void* v, void* o, float* lse, float* acc_o,
+                       float* acc_lse, int mode, int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                       float scale, fa_dtype dt, fa_stream_t stream);
+
+/*
+ * Backward contributions of one key/value chunk added into fp32 accumulators
+ * (the dK/dV and dQ kernels of fa_bwd with their epilogues adding into fp32
+ * instead of writing 16-bit gradients): with P = exp(scale Q K^T - lse) over
+ * this chunk's keys and D the rows' term from fa_bwd_preprocess (`workspace`,
+ * over the whole rows), dq_acc [B, Nq, Hq, d] += scale dS K, and dk_acc,
+ * dv_acc [B, Nk, Hkv, d] += scale dS^T Q, P^T dO (summed over each group's
+ * query heads).  Summed over a partition of the keys this is the full
+ * backward, since the chain rule is linear in the keys once LSE and D are
+ * fixed.  init bit 0: dq_acc is set instead of added to; bit 1: dk_acc and
+ * dv_acc are.  All fp32 buffers 16-byte aligned.  Otherwise as fa_bwd.
+ */
+fa_status fa_bwd_accumulate(const void* q, const void* k, const void* v, const void* dout, const float* lse,
+                            const void* workspace, float* dq_acc, float* dk_acc, float* dv_acc, int init, int B,
+                            int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale, fa_dtype dt,
+                            fa_stream_t stream);
+
+/*
  * Summation of 16-bit partial results in fp32 (the backward of the ring sums the
  * dQ, dK and dV contributions of every key/value chunk): fa_accumulate sets
  * acc[i] = (init ? 0 : acc[i]) + part[i] for n elements, fa_cast_f32 writes
@@ -300,8 +350,10 @@ fa_status fa_cast_f32(const float* acc, void* out, long long n, fa_dtype dt, fa_
 
 /*
  * Synchronises `stream`, then reads and clears the device status word that the
- * kernels set when a bounded wait runs out (FA_ERR_TIMEOUT) or a device-side
- * check fails.  Returns FA_OK when no kernel reported an error.
+ * kernels set when a bounded wait runs out (FA_ERR_TIMEOUT) or, in the checking
+ * build libfa_checks.so (same ABI, compiled with FA_CHECKS), when a device-side
+ * index check finds an access outside its tensor (FA_ERR_BOUNDS; the access is
+ * skipped, nothing traps).  Returns FA_OK when no kernel reported an error.
  */
 fa_status fa_get_device_status(fa_stream_t stream);
 

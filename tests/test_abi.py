@@ -38,11 +38,23 @@ def test_every_declared_symbol_is_exported(lib):
         assert n in _lib.SIGNATURES, f"binding lacks {n}"
 
 
+def test_checking_build_exports_the_same_boundary():
+    """libfa_checks.so (FA_CHECKS: device-side index checks) has every entry point too."""
+    from exact_io_aware_80_b200 import build
+    path = build.build(checks=True)
+    chk = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(chk, n), n
+    chk.fa_status_string.restype = ctypes.c_char_p
+    assert chk.fa_status_string(-6) == b"device-side index check failed"
+
+
 def test_status_strings_and_version(lib):
     from exact_io_aware_80_b200 import _lib
     assert _lib.fa_version() >= 1
-    for code in (0, -1, -2, -3, -4, -5):
+    for code in (0, -1, -2, -3, -4, -5, -6):
         assert _lib.status_string(code)
+        assert _lib.status_string(code) != "unknown status"
 
 
 def test_workspace_sizes(lib):
@@ -145,6 +157,13 @@ def test_fp8_entry_points_reject_bad_arguments(lib):
     assert lib.fa_fp8_quantize_qk(FAKE, FAKE, FAKE, FAKE + 2, 1, 2, 8, 128, 1, None) == -3
     assert lib.fa_fp8_quantize_v(FAKE, FAKE, FAKE, 0, 1, 2, 8, 128, 1, None) == -1
     assert lib.fa_fp8_quantize_v(FAKE, FAKE, FAKE, FAKE, 1, 2, 0, 128, 1, None) == -1
+    # q, k, v, q8, k8, v8t, qs, ks, vs, signs, ws, B, Hq, Hkv, Nq, Nk, d, dt, stream
+    qkv = [FAKE] * 9 + [0, FAKE, 1, 4, 2, 8, 8, 128, 1, None]
+    for idx, val, code in ((0, 0, -1), (10, 0, -1), (12, 5, -1), (16, 96, -2), (17, 7, -2), (3, FAKE + 8, -3),
+                           (6, FAKE + 2, -3), (9, FAKE + 2, -3), (14, 0, -1)):
+        bad = list(qkv)
+        bad[idx] = val
+        assert lib.fa_fp8_quantize_qkv(*bad) == code, (idx, val)
     # q8, qs, k8, ks, v8t, vs, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, rotated, dt, stream
     base = [FAKE] * 8 + [1, 4, 2, 8, 8, 128, 0, 0.1, 0, 1, None]
     bad = list(base)

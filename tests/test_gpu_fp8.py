@@ -62,6 +62,22 @@ def test_quantize_v_bit_exact(fa, Nk):
     assert np.array_equal(v8t.cpu().numpy(), c_ref)
 
 
+@pytest.mark.parametrize("d,dt,rotate,Nq,Nk", [(128, torch.bfloat16, True, 300, 1000), (64, torch.float16, False, 77, 129),
+                                               (128, torch.float16, False, 1, 16), (64, torch.bfloat16, True, 513, 257)])
+def test_quantize_qkv_fused_bit_exact(fa, d, dt, rotate, Nq, Nk):
+    """The fused Q+K+V quantizer gives the oracle's codes and scales bit for bit."""
+    q, k, v = workloads.make_inputs(2, 4, 2, Nq, Nk, d, dt, seed_base=7250 + Nq)
+    signs = workloads.rotation_signs(d, 7299) if rotate else None
+    q8, qs, k8, ks, v8t, vs = fa.fp8_quantize_qkv(q.cuda(), k.cuda(), v.cuda(), None if signs is None else signs.cuda())
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    sg = None if signs is None else npf(signs)
+    for got, gs, ref in ((q8, qs, f8.quantize_qk(npf(q), sg)), (k8, ks, f8.quantize_qk(npf(k), sg)),
+                         (v8t, vs, f8.quantize_v(npf(v)))):
+        assert np.array_equal(gs.cpu().numpy(), ref[1])
+        assert np.array_equal(got.cpu().numpy(), ref[0])
+
+
 def check_fwd(fa, q, k, v, causal, rotate, heads_rows, seed, out_dtype=torch.bfloat16):
     d = q.shape[-1]
     scale = 1.0 / math.sqrt(d)

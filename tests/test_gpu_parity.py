@@ -143,6 +143,26 @@ def test_bwd_small(fa, B, Hq, Hkv, Nq, Nk, d, dt, causal):
     assert rel_l2(dv, DV) <= GRAD_TOL
 
 
+@pytest.mark.parametrize("B,H,N,d,dt", [(2, 3, 333, 128, "bf16"), (1, 5, 77, 64, "fp16"), (3, 2, 1, 128, "fp16"),
+                                         (1, 32, 8192, 128, "bf16")])
+def test_bwd_preprocess_rowsum(fa, B, H, N, d, dt):
+    """D = rowsum(dO * O) from fa_bwd_preprocess against the oracle's definition.  The
+    kernel sums d exact products in fp32, so |error| <= d * 2^-24 * sum_c |dO_c O_c|
+    (the recursive-summation bound; 2^-23 leaves a factor 2 of margin)."""
+    from exact_io_aware_80_b200 import _lib
+    o, _, _, do = workloads.make_inputs(B, H, H, N, N, d, dtype_of(dt), seed_base=31 * N + d, with_do=True)
+    od, dod = o.cuda(), do.cuda()
+    ws = torch.full((B * H * N,), float("nan"), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    _lib.fa_bwd_preprocess(0, 0, 0, od.data_ptr(), dod.data_ptr(), 0, 0, 0, 0, ws.data_ptr(), B, H, H, N, N, d, 0,
+                           1.0, _lib.FA_BF16 if dt == "bf16" else _lib.FA_FP16, stream)
+    torch.cuda.synchronize()
+    Dref = oracle.bwd_preprocess(f64(o), f64(do))
+    Dg = ws.view(B, H, N).cpu().numpy().astype(np.float64)
+    Sabs = np.einsum("bihc,bihc->bhi", np.abs(f64(do)), np.abs(f64(o)))
+    assert np.all(np.abs(Dg - Dref) <= d * 2.0 ** -23 * Sabs)
+
+
 def test_bwd_gqa_training_sampled_groups(fa):
     """B=1, Hq=32, Hkv=8, N=8192 causal: KV groups 0 and 7 (their dK, dV and the
     dQ of their 4 query heads each) against the oracle."""

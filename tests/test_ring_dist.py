@@ -28,39 +28,37 @@ def _free_port():
 
 
 class OracleOps:
-    """partial = oracle attention of one chunk pair; merge = oracle log-sum-exp combine."""
+    """attend = oracle attention of one chunk pair, folded into the accumulator by the
+    oracle's log-sum-exp combine (the steps the CUDA kernel fuses)."""
 
     def __init__(self, scale):
         self.scale = scale
 
-    def partial(self, q, k, v, causal):
+    def attend(self, q, k, v, causal, o_acc, lse_acc, out, lse_out, mode):
         import oracle
-        O, L = oracle.attention_fwd(q.numpy(), k.numpy(), v.numpy(), causal, self.scale)
-        return torch.from_numpy(O), torch.from_numpy(L)
-
-    def merge(self, acc, part, last):
-        import oracle
-        o_acc, lse, out, first = acc
-        o_p, l_p = part
-        if first:
-            o_new, l_new = o_p.numpy(), l_p.numpy()
+        o_p, l_p = oracle.attention_fwd(q.numpy(), k.numpy(), v.numpy(), causal, self.scale)
+        if mode == 0:
+            o_new, l_new = o_p, l_p
         else:
             B, n, H, d = o_p.shape
-            O_parts = np.stack([o_acc.double().numpy(), o_p.numpy()], axis=3)  # [B, n, H, 2, d]
-            L_parts = np.stack([lse.double().numpy(), l_p.numpy()], axis=-1)   # [B, H, n, 2]
+            O_parts = np.stack([o_acc.double().numpy(), o_p], axis=3)  # [B, n, H, 2, d]
+            L_parts = np.stack([lse_acc.double().numpy(), l_p], axis=-1)  # [B, H, n, 2]
             O_parts = O_parts.reshape(B * n, H, 2, d)
             L_parts = L_parts.transpose(0, 2, 1, 3).reshape(B * n, H, 2)
             O, L = oracle.decode_combine(O_parts, L_parts)
             o_new = O.reshape(B, n, H, d)
             l_new = L.reshape(B, n, H).transpose(0, 2, 1)
-        o_acc.copy_(torch.from_numpy(np.ascontiguousarray(o_new)))
-        lse.copy_(torch.from_numpy(np.ascontiguousarray(l_new)))
-        if last:
-            out.copy_(o_acc)
+        o_new = torch.from_numpy(np.ascontiguousarray(o_new))
+        l_new = torch.from_numpy(np.ascontiguousarray(l_new))
+        if mode != 2:
+            o_acc.copy_(o_new)
+            lse_acc.copy_(l_new)
+        out.copy_(o_new)
+        lse_out.copy_(l_new)
 
 
 class OracleBwdOps:
-    """The backward's compute from the oracle: D, per-chunk-pair partial gradients, fp32 sums."""
+    """The backward's compute from the oracle: D, per-chunk-pair partial gradients added into fp64 sums."""
 
     def __init__(self, scale):
         self.scale = scale
@@ -69,17 +67,15 @@ class OracleBwdOps:
         import oracle
         return torch.from_numpy(oracle.bwd_preprocess(o.numpy(), do.numpy()))
 
-    def partial_bwd(self, q, k, v, o, do, lse, dvec, causal):
+    def accumulate_bwd(self, q, k, v, do, lse, dvec, causal, dq_acc, dk_acc, dv_acc, init_q, init_kv):
         import oracle
-        parts = oracle.attention_bwd_partial(q.numpy(), k.numpy(), v.numpy(), do.numpy(), lse.numpy(), dvec.numpy(),
-                                             causal, self.scale)
-        return tuple(torch.from_numpy(x) for x in parts)
-
-    def accumulate(self, acc, part, init):
-        if init:
-            acc.copy_(part)
-        else:
-            acc.add_(part)
+        dq, dk, dv = (torch.from_numpy(x) for x in oracle.attention_bwd_partial(
+            q.numpy(), k.numpy(), v.numpy(), do.numpy(), lse.numpy(), dvec.numpy(), causal, self.scale))
+        for acc, part, init in ((dq_acc, dq, init_q), (dk_acc, dk, init_kv), (dv_acc, dv, init_kv)):
+            if init:
+                acc.copy_(part)
+            else:
+                acc.add_(part)
 
     def cast(self, acc, out):
         out.copy_(acc)
