@@ -17,9 +17,11 @@ namespace {
 // each of 32 / (D / 8) rows per load; each thread takes kRowsPerThread rows of one
 // (b, h), consecutive query positions, and issues all of their loads before any
 // arithmetic so that every thread has 2 * kRowsPerThread 16-byte loads in flight.
-// Rows are ordered (b, h, i) with i fastest, so the D values a warp writes are
-// contiguous.
-constexpr int kRowsPerThread = 4;
+// A warp's rows are consecutive positions i of one (b, h), so the D values it writes
+// are contiguous; consecutive warps take consecutive heads at the same positions, so
+// the warps in flight together read neighbouring memory (position i of every head is
+// one contiguous stretch of O and dO).
+constexpr int kRowsPerThread = 8;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs p) {
@@ -29,12 +31,14 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs p) {
   const int lane = threadIdx.x & 31;
   const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int part = lane % TPR, sub = lane / TPR;
-  const long NqPad = (long)(p.Nq + WROWS - 1) / WROWS * WROWS;  // each warp stays inside one (b, h)
-  const long bh = warp * WROWS / NqPad;
-  if (bh >= (long)p.B * p.Hq) return;
-  const int i0 = (int)(warp * WROWS - bh * NqPad);
-  const long bb = bh / p.Hq;
-  const int h = (int)(bh % p.Hq);
+  const long groups = (p.Nq + WROWS - 1) / WROWS;  // position groups per (b, h)
+  const long BH = (long)p.B * p.Hq;
+  if (warp >= BH * groups) return;
+  const long bb = warp / (groups * p.Hq);  // batch, then position group, then head (fastest)
+  const long rest = warp % (groups * p.Hq);
+  const int h = (int)(rest % p.Hq);
+  const int i0 = (int)(rest / p.Hq) * WROWS;
+  const long bh = bb * p.Hq + h;
   uint4 o[kRowsPerThread], g[kRowsPerThread];
 #pragma unroll
   for (int k = 0; k < kRowsPerThread; ++k) {

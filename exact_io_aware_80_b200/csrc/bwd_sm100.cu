@@ -666,8 +666,8 @@ __global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
         if (!mbar_wait(bar(L::kBarVFull + j % L::kVStages), (j / L::kVStages) & 1, abort_flag, p.status)) return false;
         tc_fence_after();
         kmajor(kColDP, sDO, sV(j));
-        mma_commit(bar(L::kBarDP));
-        mma_commit(bar(L::kBarVEmpty + j % L::kVStages));
+        mma_commit(bar(L::kBarDP));  // without dropout this also frees V of tile j (see the elementwise warps)
+        if constexpr (DROP) mma_commit(bar(L::kBarVEmpty + j % L::kVStages));  // one V stage: free it at once
         return true;
       };
       bool ok = mbar_wait(bar(L::kBarQ), 0, abort_flag, p.status);
@@ -764,6 +764,12 @@ __global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
       }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), j & 1, abort_flag, p.status));
       if (!ok) break;
+      if (!DROP && tid == 0) {
+        // dP of tile j is complete, so its V stage (read by no other MMA) is free: this arrival
+        // stands in for an MMA commit per key tile.  With two V stages the next load into it has
+        // a tile of slack; the dropout variant's single V stage is freed by the commit instead.
+        mbar_arrive(bar(L::kBarVEmpty + j % L::kVStages));
+      }
       tc_fence_after();
       uint32_t keep[4] = {0u, 0u, 0u, 0u};  // dropout: bit cc = (this query, key kb + cc) kept
       if constexpr (DROP) {

@@ -46,18 +46,64 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
 }
 
 // In-place unnormalised Walsh-Hadamard transform of y[0..D), fp32 butterflies
-// in the order h = 1, 2, 4, ..., D / 2.
+// (a, b) -> (a + b, a - b) in the order h = 1, 2, 4, ..., D / 2.  From h = 2 on, the
+// butterflies of elements i and i + 1 run as one packed f32x2 instruction each
+// (a - b as the fused a + (-1) b: the product is exact, so it rounds once, as a
+// subtraction does).
 template <int D>
 __device__ __forceinline__ void fwht(float (&y)[D]) {
 #pragma unroll
-  for (int h = 1; h < D; h *= 2)
+  for (int i = 0; i < D; i += 2) {
+    const float a = y[i], b = y[i + 1];
+    y[i] = __fadd_rn(a, b);
+    y[i + 1] = __fsub_rn(a, b);
+  }
 #pragma unroll
-    for (int i = 0; i < D; ++i)
+  for (int h = 2; h < D; h *= 2)
+#pragma unroll
+    for (int i = 0; i < D; i += 2)
       if ((i & h) == 0) {
-        const float a = y[i], b = y[i + h];
-        y[i] = __fadd_rn(a, b);
-        y[i + h] = __fsub_rn(a, b);
+        const float2 a = make_float2(y[i], y[i + 1]), b = make_float2(y[i + h], y[i + h + 1]);
+        const float2 sum = __fadd2_rn(a, b), dif = __ffma2_rn(b, make_float2(-1.f, -1.f), a);
+        y[i] = sum.x;
+        y[i + 1] = sum.y;
+        y[i + h] = dif.x;
+        y[i + h + 1] = dif.y;
       }
+}
+
+// y / s correctly rounded to fp32, for one divisor and many dividends, without a division per
+// element: r = RN(1 / s), q1 = RN(y r), then one correction q = q1 + (y - q1 s) r with fused
+// multiply-adds.  With r correctly rounded and q1 within an ulp of y / s, the corrected quotient
+// is RN(y / s) (Markstein's theorem for FMA-based division), provided no intermediate leaves
+// the normal range, which holds for 2^-90 <= s <= 2^90 whenever |y / s| >= 2^-11; other divisors
+// take the IEEE division.  Smaller quotients may come out inexact, but every value below 2^-10
+// has the E4M3 code +-0 (the smallest code, 2^-9, takes values from 2^-10 up), and q keeps y's
+// sign, which q1 carries: the only case where the correction can flip it is y = -0 (q1 = -0,
+// q = +0), so q1's sign bit is OR-ed into q.  The choice between the two forms is made once per
+// block by the caller (div2<true> or div2<false>), so that the per-element code has no branch.
+struct Divider {
+  float s, r;
+  bool fast;
+  template <bool FAST>
+  __device__ __forceinline__ float2 div2(float2 y) const {
+    if constexpr (!FAST) {
+      return make_float2(__fdiv_rn(y.x, s), __fdiv_rn(y.y, s));
+    } else {
+      const float2 q1 = __fmul2_rn(y, make_float2(r, r));
+      const float2 e = __ffma2_rn(q1, make_float2(-s, -s), y);
+      const float2 q = __ffma2_rn(e, make_float2(r, r), q1);
+      return make_float2(__int_as_float(__float_as_int(q.x) | (__float_as_int(q1.x) & 0x80000000)),
+                         __int_as_float(__float_as_int(q.y) | (__float_as_int(q1.y) & 0x80000000)));
+    }
+  }
+};
+__device__ __forceinline__ Divider make_divider(float s) {
+  Divider d;
+  d.s = s;
+  d.r = __frcp_rn(s);
+  d.fast = s >= 0x1p-90f && s <= 0x1p90f;
+  return d;
 }
 
 // Block maximum of v over the CTA's 128 threads.
@@ -98,14 +144,6 @@ __device__ __forceinline__ void issue_rows(const T* x, uint8_t* st, int N, int H
     cp_async16(base + r * S::kRowBytes + 16 * c, src, ok);
   }
 }
-template <typename T, int D>
-__device__ __forceinline__ void stage_rows(const T* x, uint8_t* st, int N, int H, int b, int h, int n0) {
-  issue_rows<T, D>(x, st, N, H, b, h, n0);
-  cp_async_commit();
-  cp_async_wait<0>();
-  __syncthreads();
-}
-
 // Row r of the stage as fp32.
 template <typename T, int D>
 __device__ __forceinline__ void read_row(const uint8_t* st, int r, float (&y)[D]) {
@@ -123,6 +161,23 @@ __device__ __forceinline__ void read_row(const uint8_t* st, int r, float (&y)[D]
   }
 }
 
+// E4M3 codes of one row y / s, 16 at a time into row[0 .. D / 16).
+template <int D, bool FAST>
+__device__ __forceinline__ void encode_row(const float (&y)[D], const Divider& dv, uint4* row) {
+#pragma unroll
+  for (int i = 0; i < D / 16; ++i) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c = 16 * i + 4 * k;
+      const float2 lo = dv.div2<FAST>(make_float2(y[c], y[c + 1]));
+      const float2 hi = dv.div2<FAST>(make_float2(y[c + 2], y[c + 3]));
+      w[k] = (uint32_t)e4m3x2(lo.x, lo.y) | ((uint32_t)e4m3x2(hi.x, hi.y) << 16);
+    }
+    row[i] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 // One 128-row block of Q or K: (signs, Walsh-Hadamard), block amax, scale, E4M3 codes.
 template <typename T, int D>
 __device__ __forceinline__ void quant_rows_block(const QuantJob& job, const float* signs, int j, int h, int b, int B,
@@ -131,32 +186,37 @@ __device__ __forceinline__ void quant_rows_block(const QuantJob& job, const floa
   const int r = threadIdx.x;
   float y[D];
   read_row<T, D>(st, r, y);
-  if (signs) {
+  if (signs) {  // the rotation signs, staged in shared memory by the kernel
+    const float4* s4 = reinterpret_cast<const float4*>(signs);
 #pragma unroll
-    for (int i = 0; i < D; ++i) y[i] = y[i] * signs[i];  // exact: +-1
+    for (int i = 0; i < D / 4; ++i) {
+      const float4 g = s4[i];
+      const float2 a = __fmul2_rn(make_float2(y[4 * i], y[4 * i + 1]), make_float2(g.x, g.y));  // exact: +-1
+      const float2 c = __fmul2_rn(make_float2(y[4 * i + 2], y[4 * i + 3]), make_float2(g.z, g.w));
+      y[4 * i] = a.x;
+      y[4 * i + 1] = a.y;
+      y[4 * i + 2] = c.x;
+      y[4 * i + 3] = c.y;
+    }
     fwht<D>(y);
   }
-  float amax = 0.f;
+  float am[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll
-  for (int i = 0; i < D; ++i) amax = fmaxf(amax, fabsf(y[i]));
+  for (int i = 0; i < D; i += 4)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) am[k] = fmaxf(am[k], fabsf(y[i + k]));
+  float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
   amax = block_max(amax, red);  // its barriers also order every read of the stage before the writes below
   const float s = scale_of(amax);
   if (r == 0 && FA_IN_BOUNDS(status, ((long)b * job.H + h) * job.nblk + j, (long)B * job.H * job.nblk))
     job.scales[((long)b * job.H + h) * job.nblk + j] = s;
+  const Divider dv = make_divider(s);
   // codes of row r over the first D bytes of its own stage row
   uint4* row = reinterpret_cast<uint4*>(st + r * S::kRowBytes);
-#pragma unroll
-  for (int i = 0; i < D / 16; ++i) {
-    uint32_t w[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int c = 16 * i + 4 * k;
-      const uint32_t lo = e4m3x2(__fdiv_rn(y[c], s), __fdiv_rn(y[c + 1], s));
-      const uint32_t hi = e4m3x2(__fdiv_rn(y[c + 2], s), __fdiv_rn(y[c + 3], s));
-      w[k] = lo | (hi << 16);
-    }
-    row[i] = make_uint4(w[0], w[1], w[2], w[3]);
-  }
+  if (dv.fast)
+    encode_row<D, true>(y, dv, row);
+  else
+    encode_row<D, false>(y, dv, row);
   __syncthreads();
   // D code bytes per row, 16 at a time, consecutive threads on consecutive chunks of a row
   constexpr int C8 = D / 16;
@@ -177,10 +237,12 @@ __device__ __forceinline__ void v_amax_block(const QuantJob& job, int j, int h, 
                                              float* red, int* status) {
   float y[D];
   read_row<T, D>(st, threadIdx.x, y);
-  float amax = 0.f;
+  float am[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int i = 0; i < D; ++i) amax = fmaxf(amax, fabsf(y[i]));
-  amax = block_max(amax, red);
+  for (int i = 0; i < D; i += 4)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) am[k] = fmaxf(am[k], fabsf(y[i + k]));
+  const float amax = block_max(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])), red);
   if (threadIdx.x == 0 && FA_IN_BOUNDS(status, ((long)b * job.H + h) * job.nblk + j, (long)B * job.H * job.nblk))
     job.scales[((long)b * job.H + h) * job.nblk + j] = amax;
 }
@@ -213,7 +275,11 @@ __global__ void __launch_bounds__(kRows) quant_kernel(QuantJobs jobs, const floa
                                                       long total) {
   extern __shared__ __align__(16) uint8_t q_smem[];  // two stages
   __shared__ float red[4];
+  __shared__ __align__(16) float s_signs[D];
   uint8_t* stage[2] = {q_smem, q_smem + Stage<D>::kBytes};
+  if (signs)
+    for (int i = threadIdx.x; i < D; i += kRows) s_signs[i] = signs[i];
+  const float* sg = signs ? s_signs : nullptr;  // visible to every thread after the loop's first barrier
   long id = blockIdx.x;
   if (id < total) issue_block<T, D>(jobs, block_ref(jobs, id, B), stage[0]);
   cp_async_commit();
@@ -226,12 +292,43 @@ __global__ void __launch_bounds__(kRows) quant_kernel(QuantJobs jobs, const floa
     const BlockRef r = block_ref(jobs, id, B);
     const QuantJob& job = jobs.job[r.job];
     if (job.kind == kQuantRows)
-      quant_rows_block<T, D>(job, signs, r.j, r.h, r.b, B, stage[it & 1], red, jobs.status);
+      quant_rows_block<T, D>(job, sg, r.j, r.h, r.b, B, stage[it & 1], red, jobs.status);
     else
       v_amax_block<T, D>(job, r.j, r.h, r.b, B, stage[it & 1], red, jobs.status);
     __syncthreads();  // every thread is done with this buffer before it is refilled
   }
   cp_async_wait<0>();
+}
+
+// Codes of a staged V block, transposed: thread t takes the column pair (2p, 2p + 1),
+// p = t mod (D / 2), over the keys [K g, K g + K) with g = t div (D / 2) and K = 128 / (128 / (D / 2))
+// = D / 2 keys; one 32-bit shared-memory read gives both columns of a key (rows past Nk were
+// staged as zeros).  Code row c of out holds the 128 keys of column c (kRows + 16 bytes per row).
+template <typename T, int D, bool FAST>
+__device__ __forceinline__ void encode_columns(const uint8_t* st, uint8_t* out, const Divider& dv) {
+  using S = Stage<D>;
+  constexpr int kOutRow = kRows + 16;
+  constexpr int P = D / 2, K = P;
+  static_assert(kRows % P == 0 && (kRows / P) * K == kRows, "column pairs x key groups = threads");
+  const int p = threadIdx.x % P, g = threadIdx.x / P;
+#pragma unroll 2
+  for (int k16 = 0; k16 < K / 16; ++k16) {
+    const int key0 = K * g + 16 * k16;
+    uint32_t w0[4], w1[4];  // codes of column 2p and 2p + 1
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float2 f[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        f[e] = Elem<T>::unpack(*reinterpret_cast<const uint32_t*>(st + (key0 + 4 * q + e) * S::kRowBytes + 4 * p));
+      const float2 a0 = dv.div2<FAST>(make_float2(f[0].x, f[1].x)), b0 = dv.div2<FAST>(make_float2(f[2].x, f[3].x));
+      const float2 a1 = dv.div2<FAST>(make_float2(f[0].y, f[1].y)), b1 = dv.div2<FAST>(make_float2(f[2].y, f[3].y));
+      w0[q] = (uint32_t)e4m3x2(a0.x, a0.y) | ((uint32_t)e4m3x2(b0.x, b0.y) << 16);
+      w1[q] = (uint32_t)e4m3x2(a1.x, a1.y) | ((uint32_t)e4m3x2(b1.x, b1.y) << 16);
+    }
+    *reinterpret_cast<uint4*>(out + (2 * p) * kOutRow + key0) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+    *reinterpret_cast<uint4*>(out + (2 * p + 1) * kOutRow + key0) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+  }
 }
 
 // One 128-key block of V: the head's scale from the block maxima, then codes written
@@ -247,32 +344,23 @@ __global__ void __launch_bounds__(kRows) v_quant_kernel(const T* __restrict__ v,
   uint8_t* out = vq_smem + S::kBytes;
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int nb = gridDim.x;
-  stage_rows<T, D>(v, st, Nk, H, b, h, j * kRows);
+  __shared__ float red[4];
+  issue_rows<T, D>(v, st, Nk, H, b, h, j * kRows);
+  cp_async_commit();
+  // the head's amax over its block maxima, while the block's copies are in flight
   float amax = 0.f;
   const float* ph = part + ((long)b * H + h) * nb;
-  for (int i = 0; i < nb; ++i) amax = fmaxf(amax, ph[i]);
+  for (int i = threadIdx.x; i < nb; i += kRows) amax = fmaxf(amax, ph[i]);
+  amax = block_max(amax, red);
+  cp_async_wait<0>();
+  __syncthreads();
   const float s = scale_of(amax);
   if (j == 0 && threadIdx.x == 0 && FA_IN_BOUNDS(status, (long)b * H + h, (long)gridDim.z * H)) scale[(long)b * H + h] = s;
-  // thread c < D encodes column c of the block: keys 0..127 (rows past Nk were staged as zeros)
-  for (int c = threadIdx.x; c < D; c += kRows) {
-#pragma unroll 2
-    for (int k16 = 0; k16 < kRows / 16; ++k16) {
-      uint32_t w[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float f[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int key = 16 * k16 + 4 * q + e;
-          const uint16_t raw = *reinterpret_cast<const uint16_t*>(st + key * S::kRowBytes + 2 * c);
-          f[e] = Elem<T>::unpack((uint32_t)raw).x;
-        }
-        w[q] = (uint32_t)e4m3x2(__fdiv_rn(f[0], s), __fdiv_rn(f[1], s)) |
-               ((uint32_t)e4m3x2(__fdiv_rn(f[2], s), __fdiv_rn(f[3], s)) << 16);
-      }
-      *reinterpret_cast<uint4*>(out + c * kOutRow + 16 * k16) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-  }
+  const Divider dv = make_divider(s);
+  if (dv.fast)
+    encode_columns<T, D, true>(st, out, dv);
+  else
+    encode_columns<T, D, false>(st, out, dv);
   __syncthreads();
   // row c of the block: keys 128 j .. 128 j + 127, clipped to Npad (a multiple of 16); codes of
   // keys past Nk are zeros

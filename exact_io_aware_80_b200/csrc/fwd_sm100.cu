@@ -11,7 +11,10 @@
 // threads = 3 warpgroups) walks the (row block, head, batch) work tiles,
 // longest causal row blocks first; the next tile's Q/K/V loads and first
 // score MMAs overlap the current tile's epilogue.  Per work tile:
-//   * two 128-row query tiles Q0, Q1 share every K/V tile the CTA loads;
+//   * two 128-row query tiles Q0, Q1 share every K/V tile the CTA loads: 256
+//     consecutive rows of one head, or (causal or block-sparse GQA with an even
+//     group) the same 128 rows of two heads of one KV group, whose key ranges
+//     then coincide;
 //   * warp 8 (one thread) issues TMA loads: Q0/Q1 once, then 128-key K and V
 //     tiles into a two-stage shared-memory ring (128-byte swizzle);
 //   * warp 9 (one thread) issues the tcgen05 MMAs: S_t = Q_t K_j^T into TMEM
@@ -88,16 +91,17 @@ struct Smem {
   static constexpr int kPanel = 128 * 128;  // one [128 rows][128 bytes] swizzled panel
   // a Q, K or V tile: 16-bit [128][D] as D / 64 panels, or E4M3 [128][D = 128] as one panel
   static constexpr int kTile = F8 ? 128 * D : (D / 64) * kPanel;
-  static constexpr int kTileOut = (D / 64) * kPanel;  // a 16-bit O tile
+  static constexpr int kStageBytes = 2 * kPanel;  // one 64-column O panel per query tile
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kTiles * kTile;
   static constexpr int kOffV = kOffK + kStages * kTile;
-  static constexpr int kOffStage = kOffV + kStages * kTile;  // one 16-bit O tile on its way to a TMA store
-  static constexpr int kOffBar = kOffStage + kTileOut;
+  static constexpr int kOffStage = kOffV + kStages * kTile;  // two 16 KB halves, one per query tile: O panels
+                                                             // on their way to a TMA store
+  static constexpr int kOffBar = kOffStage + kStageBytes;
   // kBarQ/kBarQEmpty: the query tiles of a work tile landed / may be replaced; kBarO + t: tile t's
   // last PV finished; kBarOFree + t: the epilogue of tile t has read O_t from TMEM;
-  // kBarStageFull + t: tile t's rows are in the stage buffer; kBarStageDone + t: the TMA store of
-  // tile t has read the stage buffer (the two tiles take turns with it)
+  // kBarStageFull + t: a panel of tile t's rows is in tile t's half of the stage buffer;
+  // kBarStageDone + t: the TMA store of that panel has read it
   enum { kBarQ = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7, kBarS = 9, kBarP = 11, kBarO = 13,
          kBarDrain = 15, kBarQEmpty = 16, kBarOFree = 17, kBarStageFull = 19, kBarStageDone = 21, kNumBars = 23 };
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
@@ -112,8 +116,9 @@ struct Params {
   int B, Hq, Hkv, Nq, Nk;
   float scale_log2;
   int* status;
-  int num_mblk;  // 256-row blocks per (b, h)
-  int num_work;  // num_mblk * Hq * B work tiles
+  int num_mblk;  // row units per (b, head unit): 256 rows, or 128 with paired heads
+  int num_work;  // num_mblk * head units * B work tiles
+  int pair;      // 1: the two query tiles are heads h, h + 1 (one KV group) over the same 128 rows
   // FP8 only: Q / K scales per 128-row block ([B,Hq,nqb], [B,Hkv,nkb]), V scale per head [B,Hkv]
   const float* q_scale;
   const float* k_scale;
@@ -176,20 +181,29 @@ __device__ __forceinline__ void merge_acc_row(const Params& p, long orow, long l
 // w = k G + i on even rounds and k G + (G - 1 - i) on odd ones, which balances
 // the decreasing tile lengths across SMs (work_index below).
 struct Work {
-  int mblk, hq, b;
+  int mblk, hq, b;  // row unit, first query head, batch
 };
+// The two query tiles of a work tile: rows 256 mblk .. + 255 of head hq (tile t: 128 rows at
+// 256 mblk + 128 t), or, with paired heads, rows 128 mblk .. + 127 of heads hq and hq + 1, which
+// share one KV head (GQA groups of even size) and so need exactly the same K/V tiles -- no key
+// tile is computed for one query tile and masked away for the other.
+__device__ __forceinline__ int tile_row(const Params& p, const Work& x, int t) {
+  return p.pair ? x.mblk * kBM : x.mblk * (kTiles * kBM) + t * kBM;
+}
+__device__ __forceinline__ int tile_head(const Params& p, const Work& x, int t) { return x.hq + (p.pair ? t : 0); }
 __device__ __forceinline__ int work_index(int round) {
   const int G = gridDim.x, i = blockIdx.x;
   return round * G + ((round & 1) ? (G - 1 - i) : i);
 }
 template <bool CAUSAL>
 __device__ __forceinline__ Work work_at(const Params& p, int w) {
-  const int per_len = p.Hq * p.B;
+  const int hunits = p.pair ? p.Hq / 2 : p.Hq;
+  const int per_len = hunits * p.B;
   const int r = w / per_len, rest = w % per_len;
   Work x;
   x.mblk = CAUSAL ? p.num_mblk - 1 - r : r;
-  x.hq = rest % p.Hq;
-  x.b = rest / p.Hq;
+  x.hq = (rest % hunits) * (p.pair ? 2 : 1);
+  x.b = rest / hunits;
   return x;
 }
 
@@ -207,17 +221,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int off = p.Nk - p.Nq;
-  auto blocks_of = [&](int mblk) {  // K/V tiles a row block visits (causal rows stop at their diagonal)
-    const int m0 = mblk * (kTiles * kBM);
-    const int n_end = CAUSAL ? min(p.Nk, m0 + kTiles * kBM + off) : p.Nk;
+  auto blocks_of = [&](const Work& x) {  // K/V tiles a work tile visits (causal rows stop at their diagonal)
+    const int rows_end = (x.mblk + 1) * (p.pair ? kBM : kTiles * kBM);
+    const int n_end = CAUSAL ? min(p.Nk, rows_end + off) : p.Nk;
     return (n_end + kBN - 1) / kBN;
   };
   // block-sparse: the table row of query tile t of a work tile (null past Nq), and the first
   // K/V tile >= j below nblk that either query tile marks (j itself for dense attention)
   auto mask_row = [&](const Work& x, int t) -> const uint8_t* {
-    const int qb = kTiles * x.mblk + t;
+    const int qb = tile_row(p, x, t) / kBM;
     if (qb >= p.nqb) return nullptr;
-    const long mi = (((long)x.b * p.Hq + x.hq) * p.nqb + qb) * p.nkb;
+    const long mi = (((long)x.b * p.Hq + tile_head(p, x, t)) * p.nqb + qb) * p.nkb;
     if (!FA_IN_BOUNDS(p.status, mi + p.nkb - 1, (long)p.B * p.Hq * p.nqb * p.nkb)) return nullptr;
     return p.block_mask + mi;
   };
@@ -267,8 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int wl = 0, w = work_index(0); w < p.num_work; w = work_index(++wl)) {
         const Work x = work_at<CAUSAL>(p, w);
         const int hk = x.hq / (p.Hq / p.Hkv);
-        const int m0 = x.mblk * (kTiles * kBM);
-        const int nblk = blocks_of(x.mblk);
+        const int nblk = blocks_of(x);
         if constexpr (SPARSE) {
           if (next_vis(x, 0, nblk) >= nblk) continue;  // nothing to load: the softmax warps write zeros
         } else {
@@ -280,12 +293,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int t = 0; t < kTiles; ++t) {
           if constexpr (F8) {
-            tma_load_4d(sb + L::kOffQ + t * L::kTile, &tmQ, bar(L::kBarQ), 0, x.hq, m0 + t * kBM, x.b);
+            tma_load_4d(sb + L::kOffQ + t * L::kTile, &tmQ, bar(L::kBarQ), 0, tile_head(p, x, t), tile_row(p, x, t),
+                        x.b);
           } else {
 #pragma unroll
             for (int pn = 0; pn < D / 64; ++pn)
-              tma_load_4d(sb + L::kOffQ + t * L::kTile + pn * L::kPanel, &tmQ, bar(L::kBarQ), 64 * pn, x.hq,
-                          m0 + t * kBM, x.b);
+              tma_load_4d(sb + L::kOffQ + t * L::kTile + pn * L::kPanel, &tmQ, bar(L::kBarQ), 64 * pn,
+                          tile_head(p, x, t), tile_row(p, x, t), x.b);
           }
         }
         last_q = we++;
@@ -381,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int we = 0;  // work tiles with at least one K/V tile so far
       for (int wl = 0, w = work_index(0); ok && w < p.num_work; w = work_index(++wl)) {
         const Work x = work_at<CAUSAL>(p, w);
-        const int nblk = blocks_of(x.mblk);
+        const int nblk = blocks_of(x);
         const int j0 = next_vis(x, 0, nblk);
         if constexpr (SPARSE) {
           if (j0 >= nblk) continue;
@@ -424,12 +438,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           pv(1, st, j == j0);
-          if (!more) mma_commit(bar(L::kBarO + 1));
-          mma_commit(bar(L::kBarVEmpty + st));
+          if (!more) {
+            mma_commit(bar(L::kBarO + 1));
+            mma_commit(bar(L::kBarVEmpty + st));  // inside a work tile the softmax warps free V (below)
+          }
           if (more) {
             qk(1, st1);
-            mma_commit(bar(L::kBarS + 1));
-            mma_commit(bar(L::kBarKEmpty + st1));
+            mma_commit(bar(L::kBarS + 1));  // also frees K of tile g + 1 and V of tile g (see the softmax)
             if (next_vis(x, jn + 1, nblk) >= nblk) mma_commit(bar(L::kBarQEmpty));  // last score MMAs issued
           }
           j = jn;
@@ -455,10 +470,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int we = 0;  // work tiles with at least one K/V tile so far
     for (int wl = 0, w = work_index(0); ok && w < p.num_work; w = work_index(++wl)) {
       const Work x = work_at<CAUSAL>(p, w);
-      const int h = x.hq, b = x.b;
-      const int m0 = x.mblk * (kTiles * kBM);
-      const int nblk = blocks_of(x.mblk);
-      const int row_first = m0 + t * kBM;
+      const int h = tile_head(p, x, t), b = x.b;
+      const int nblk = blocks_of(x);
+      const int row_first = tile_row(p, x, t);
       const int row = row_first + wq * 32 + lane;
       const int j0 = next_vis(x, 0, nblk);
       if constexpr (SPARSE) {
@@ -515,6 +529,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + t), g & 1, abort_flag, p.status));
         if (!ok) break;
+        if (t == 1 && wq == 0 && lane == 0 && j != j0) {
+          // S_1 of tile g is complete, and with it every MMA issued before it: the score MMAs
+          // of tile g (its K stage is free) and P_1 V of tile g - 1 (its V stage is free).  This
+          // arrival stands in for two MMA commits per key tile; the first tile of a work tile
+          // and the last one's V are still freed by commits.
+          mbar_arrive(bar(L::kBarKEmpty + (g & 1)));
+          mbar_arrive(bar(L::kBarVEmpty + ((g - 1) & 1)));
+        }
         tc_fence_after();
         float s[kBN];
         {
@@ -627,15 +649,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q = 0; q < D / 32; ++q) reg_fence(*reinterpret_cast<uint32_t(*)[32]>(r + 32 * q));
         tc_fence_before();
         mbar_arrive(bar(L::kBarOFree + t));
-        // the stage buffer alternates tile 0, tile 1, tile 0 (next work tile), ...
-        if (t == 1)
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarStageDone + 0), we & 1, abort_flag, p.status));
-        else if (we > 0)
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarStageDone + 1), (we - 1) & 1, abort_flag, p.status));
       }
       if (ok) {
-        // O / l as 16-bit into the stage buffer, laid out as the TMA box expects: 64-column
-        // panels of 128-byte rows, 16-byte chunk c of row r at chunk c ^ (r & 7)
         float num = 1.f;  // FP8: V's scale; dropout: 1 / (1 - p)
         if constexpr (F8) num = FA_IN_BOUNDS(p.status, (long)b * p.Hkv + hk, (long)p.B * p.Hkv) ? p.v_scale[(long)b * p.Hkv + hk] : 0.f;
         if constexpr (DROP) num = p.drop.inv_keep;
@@ -650,30 +665,40 @@ __global__ void __launch_bounds__(kThreads, 1)
               FA_IN_BOUNDS(p.status, lrow, (long)p.B * p.Hq * p.Nq))
             merge_acc_row<D>(p, orow, lrow, r, inv, lse_row);
         }
-        const int rr = wq * 32 + lane;
-        const uint32_t srow = sb + L::kOffStage + rr * 128;
-        auto o2 = [&](int i) { return Elem<T>::pack(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv); };
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c)
-          st_shared_v4(srow + (c >> 3) * L::kPanel + (((c & 7) ^ (rr & 7)) << 4), o2(8 * c), o2(8 * c + 2),
-                       o2(8 * c + 4), o2(8 * c + 6));
-        fence_proxy_async_smem();
-        mbar_arrive(bar(L::kBarStageFull + t));
         if (row < p.Nq && FA_IN_BOUNDS(p.status, ((long)b * p.Hq + h) * p.Nq + row, (long)p.B * p.Hq * p.Nq))
           p.lse[((long)b * p.Hq + h) * p.Nq + row] = lse_row;
-        if (wq == 0 && lane == 0) {
-          // one thread of the tile stores it; rows past Nq are clipped by the tensor map
-          ok = mbar_wait(bar(L::kBarStageFull + t), we & 1, abort_flag, p.status);
-          if (ok) {
+        // O / l as 16-bit, one 64-column panel at a time, through this tile's own half of the
+        // stage buffer (16 KB, laid out as the TMA box expects: 128-byte rows, 16-byte chunk c of
+        // row r at chunk c ^ (r & 7)); the two tiles' halves are separate, so their epilogues
+        // overlap.  One thread of the tile stores each panel; rows past Nq are clipped by the map.
+        const int rr = wq * 32 + lane;
+        const uint32_t half = sb + L::kOffStage + t * L::kPanel;
+        auto o2 = [&](int i) { return Elem<T>::pack(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv); };
 #pragma unroll
-            for (int pn = 0; pn < D / 64; ++pn)
-              tma_store_4d(&tmO, sb + L::kOffStage + pn * L::kPanel, 64 * pn, h, row_first, b);
-            bulk_commit();
-            bulk_wait_read_all();
-            mbar_arrive(bar(L::kBarStageDone + t));
+        for (int pn = 0; pn < D / 64; ++pn) {
+          const int u = we * (D / 64) + pn;  // uses of this tile's half so far
+          if (u > 0)
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarStageDone + t), (u - 1) & 1, abort_flag, p.status));
+          if (!ok) break;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const int cc = 8 * pn + c;
+            st_shared_v4(half + rr * 128 + ((c ^ (rr & 7)) << 4), o2(8 * cc), o2(8 * cc + 2), o2(8 * cc + 4),
+                         o2(8 * cc + 6));
           }
+          fence_proxy_async_smem();
+          mbar_arrive(bar(L::kBarStageFull + t));
+          if (wq == 0 && lane == 0) {
+            ok = mbar_wait(bar(L::kBarStageFull + t), u & 1, abort_flag, p.status);
+            if (ok) {
+              tma_store_4d(&tmO, half, 64 * pn, h, row_first, b);
+              bulk_commit();
+              bulk_wait_read_all();
+              mbar_arrive(bar(L::kBarStageDone + t));
+            }
+          }
+          ok = __all_sync(0xffffffffu, ok);
         }
-        ok = __all_sync(0xffffffffu, ok);
       }
       ++we;
     }
@@ -700,10 +725,14 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t s) {
   if (!make_map(&mq, a.q, bf16, D, a.Hq, a.Nq, a.B, kBM) || !make_map(&mk, a.k, bf16, D, a.Hkv, a.Nk, a.B, kBN) ||
       !make_map(&mv, a.v, bf16, D, a.Hkv, a.Nk, a.B, kBN) || !make_map(&mo, a.o, bf16, D, a.Hq, a.Nq, a.B, kBM))
     return cudaErrorInvalidValue;
-  const int num_mblk = (a.Nq + kTiles * kBM - 1) / (kTiles * kBM);
-  const long long num_work = (long long)num_mblk * a.Hq * a.B;
+  // paired heads for even GQA groups when the two query tiles' key ranges would differ otherwise
+  // (causal, block-sparse); non-causal dense tiles need the same keys either way
+  const int pair = ((a.Hq / a.Hkv) % 2 == 0 && (CAUSAL || a.block_mask)) ? 1 : 0;
+  const int unit = pair ? kBM : kTiles * kBM;
+  const int num_mblk = (a.Nq + unit - 1) / unit;
+  const long long num_work = (long long)num_mblk * (pair ? a.Hq / 2 : a.Hq) * a.B;
   if (num_work > (1ll << 31) - 1) return cudaErrorInvalidValue;
-  Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, a.scale * kLog2e, a.status, num_mblk, (int)num_work,
+  Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, a.scale * kLog2e, a.status, num_mblk, (int)num_work, pair,
            nullptr, nullptr, nullptr, (a.Nq + kBM - 1) / kBM, (a.Nk + kBN - 1) / kBN, a.block_mask,
            Dropout{a.drop_thr, a.drop_inv_keep, a.seed_lo, a.seed_hi, a.drop_offset}, a.acc_o, a.acc_lse, a.acc_mode};
   if (a.acc_o) {
@@ -760,11 +789,13 @@ cudaError_t launch_f8(const Fp8AttnArgs& a, cudaStream_t s) {
   if (!make_map_u8(&mq, a.q8, dq, sq, box_qk) || !make_map_u8(&mk, a.k8, dk, sk, box_qk) ||
       !make_map_u8(&mv, a.v8t, dv, sv, box_v) || !make_map(&mo, a.o, Elem<T>::kBf16, D, a.Hq, a.Nq, a.B, kBM))
     return cudaErrorInvalidValue;
-  const int num_mblk = (a.Nq + kTiles * kBM - 1) / (kTiles * kBM);
-  const long long num_work = (long long)num_mblk * a.Hq * a.B;
+  const int pair = ((a.Hq / a.Hkv) % 2 == 0 && CAUSAL) ? 1 : 0;
+  const int unit = pair ? kBM : kTiles * kBM;
+  const int num_mblk = (a.Nq + unit - 1) / unit;
+  const long long num_work = (long long)num_mblk * (pair ? a.Hq / 2 : a.Hq) * a.B;
   if (num_work > (1ll << 31) - 1) return cudaErrorInvalidValue;
   const float sl2 = a.scale * kLog2e / (a.rotated ? (float)D : 1.f);
-  Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, sl2, a.status, num_mblk, (int)num_work,
+  Params p{a.o, a.lse, a.B, a.Hq, a.Hkv, a.Nq, a.Nk, sl2, a.status, num_mblk, (int)num_work, pair,
            a.q_scale, a.k_scale, a.v_scale, (a.Nq + kBM - 1) / kBM, (a.Nk + kBN - 1) / kBN, nullptr, Dropout{},
            nullptr, nullptr, 0};
   auto kern = fwd_sm100_kernel<T, D, CAUSAL, true, false, false>;
