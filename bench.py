@@ -693,6 +693,8 @@ def run_long_context(args, torch, fa, _lib, workloads, dev, stream, world, peaks
     kname = {"fwd": "fwd_sm100_kernel", "bwd_dkdv": "bwd_dkdv_sm100_kernel", "bwd_dq": "bwd_dq_sm100_kernel"}[dom]
     ach = kflops[dom] / (per[dom] * 1e-3) / 1e12
     fwd_t, bwd_t = F / (per["fwd"] * 1e-3) / 1e12, 2.5 * F / (bwd_ms * 1e-3) / 1e12
+    traffic8192 = traffic_for(kname)
+    traffic8192 = None if traffic8192 is None else int(traffic8192 * N / 8192)
     return {"workload": f"long-context GQA step: fwd+bwd, B={B} Hq={Hq} Hkv={Hkv} Nq=Nk={N} d={d} causal bf16",
             "ms_per_step": round(ms, 4), "value": round(world * 3.5 * F / (ms * 1e-3) / 1e12, 1), "unit": "TFLOP/s",
             "fwd_ms": round(per["fwd"], 4), "fwd_tflops": round(fwd_t, 1),
@@ -701,7 +703,8 @@ def run_long_context(args, torch, fa, _lib, workloads, dev, stream, world, peaks
             "bwd_frac_of_datasheet_2250": round(bwd_t / DENSE_BF16_DATASHEET_TFLOPS, 4),
             "per_kernel_ms": {kk: round(vv, 4) for kk, vv in per.items()},
             "roofline": {"bound": "tensor", "kernel": kname, "achieved": round(ach, 1), "peak": peak,
-                         "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                         "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": traffic8192,
+                         "traffic_basis": "the N=8192 figure x N / 8192 (each input is read once per launch)",
                          "peak_source": f"{peaks_kind} {key}", "algorithmic_flops_per_launch": kflops[dom],
                          "avg_launch_ms": round(per[dom], 4)},
             "gpu_launches": 4 * K}

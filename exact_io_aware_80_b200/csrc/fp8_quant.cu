@@ -271,7 +271,7 @@ __device__ __forceinline__ void issue_block(const QuantJobs& jobs, const BlockRe
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kRows) quant_kernel(QuantJobs jobs, const float* __restrict__ signs, int B,
+__global__ void __launch_bounds__(kRows, 3) quant_kernel(QuantJobs jobs, const float* __restrict__ signs, int B,
                                                       long total) {
   extern __shared__ __align__(16) uint8_t q_smem[];  // two stages
   __shared__ float red[4];
