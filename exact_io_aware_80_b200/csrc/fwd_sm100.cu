@@ -81,6 +81,14 @@ constexpr int kThreads = 384;
 // (2 x 128 x 200 + 128 x 104 = 64512).
 constexpr int kRegsSoftmax = 200;
 constexpr int kRegsControl = 104;
+// Of every eight column pairs of a score block, how many take the FMA-pipe exponential
+// (exp2_fma2) instead of ex2.approx, with 16-bit and with FP8 operands.
+#ifndef FA_FWD_EXP2_EIGHTHS
+#define FA_FWD_EXP2_EIGHTHS 2
+#endif
+#ifndef FA_FWD_F8_EXP2_EIGHTHS
+#define FA_FWD_F8_EXP2_EIGHTHS 2
+#endif
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * 168, "register split exceeds the launch");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when m grows by more than 2^8
 __host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }        // S_t / P_t
@@ -212,6 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, Params p) {
   using L = Smem<D, F8>;
+  constexpr int kExpFma8 = F8 ? FA_FWD_F8_EXP2_EIGHTHS : FA_FWD_EXP2_EIGHTHS;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
@@ -527,6 +536,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int wd = 0; wd < 4; ++wd) keep[wd] = own[wd] | __shfl_xor_sync(0xffffffffu, other[wd], 1);
         }
+        float cj = cq;  // FP8: times the K block's scale, loaded before the scores arrive
+        if constexpr (F8) {
+          const long si = ((long)b * p.Hkv + hk) * p.nkb + j;
+          cj = FA_IN_BOUNDS(p.status, si, (long)p.B * p.Hkv * p.nkb) ? cq * p.k_scale[si] : 0.f;
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + t), g & 1, abort_flag, p.status));
         if (!ok) break;
         if (t == 1 && wq == 0 && lane == 0 && j != j0) {
@@ -557,11 +571,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             s[64 + i] = __uint_as_float(r2[i]);
             s[96 + i] = __uint_as_float(r3[i]);
           }
-        }
-        float cj = cq;  // FP8: times the K block's scale
-        if constexpr (F8) {
-          const long si = ((long)b * p.Hkv + hk) * p.nkb + j;
-          cj = FA_IN_BOUNDS(p.status, si, (long)p.B * p.Hkv * p.nkb) ? cq * p.k_scale[si] : 0.f;
         }
         const int kbase = j * kBN;
         bool on = true;  // block-sparse: this query tile computes block (., j)
@@ -595,8 +604,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             const int c0 = 64 * half + 2 * i;
-            const float2 a = exp2_pair(__ffma2_rn(make_float2(s[c0], s[c0 + 1]), c2, nm2), 32 * half + i);
-            const float2 bb = exp2_pair(__ffma2_rn(make_float2(s[c0 + 2], s[c0 + 3]), c2, nm2), 32 * half + i + 1);
+            const float2 a = exp2_pair8<kExpFma8>(__ffma2_rn(make_float2(s[c0], s[c0 + 1]), c2, nm2), 32 * half + i);
+            const float2 bb =
+                exp2_pair8<kExpFma8>(__ffma2_rn(make_float2(s[c0 + 2], s[c0 + 3]), c2, nm2), 32 * half + i + 1);
             rs0 = __fadd2_rn(rs0, a);
             rs1 = __fadd2_rn(rs1, bb);
             float2 ad = a, bd = bb;  // the weights of the P V product

@@ -291,6 +291,15 @@ __device__ __forceinline__ float2 exp2_pair(float2 x, int pair) {
   return make_float2(ex2(x.x), ex2(x.y));
 }
 
+// The same with the share in eighths: K of every 8 consecutive column pairs, spread evenly
+// (pair p takes the FMA form when floor((p + 1) K / 8) > floor(p K / 8); K = 2 picks pairs
+// 3 and 7 of every 8, as exp2_pair with one pair in four).
+template <int K>
+__device__ __forceinline__ float2 exp2_pair8(float2 x, int pair) {
+  if (((pair + 1) * K) / 8 != (pair * K) / 8) return exp2_fma2(x);
+  return make_float2(ex2(x.x), ex2(x.y));
+}
+
 // Bounded wait that ignores the abort flag (used while draining on the error path).
 __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, int* status) {
   volatile int never = 0;
