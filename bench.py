@@ -207,20 +207,29 @@ def run_ours(args):
         _lib.fa_fwd(ptrs[0], ptrs[1], ptrs[2], ptrs[3], ptrs[5], B, Hq, Hkv, N, N, d, 1, w.scale, dt, sh)
 
     def step(ev=None):
+        """The training step as a user runs it: fa_fwd, then fa_bwd (preprocess, dK/dV, and dQ
+        launched as a programmatic dependent of dK/dV, so it fills the SMs dK/dV's tail frees)."""
         if ev:
             ev[0].record(stream)
         fwd()
         if ev:
             ev[1].record(stream)
-        _lib.fa_bwd_preprocess(*bargs)
+        _lib.fa_bwd(*bargs)
         if ev:
             ev[2].record(stream)
+
+    def step_per_kernel(ev):
+        """The same launches one entry point at a time, with an event between every two: the
+        per-kernel durations behind the roofline (dQ here starts after dK/dV has finished)."""
+        ev[0].record(stream)
+        fwd()
+        ev[1].record(stream)
+        _lib.fa_bwd_preprocess(*bargs)
+        ev[2].record(stream)
         _lib.fa_bwd_dkdv(*bargs)
-        if ev:
-            ev[3].record(stream)
+        ev[3].record(stream)
         _lib.fa_bwd_dq(*bargs)
-        if ev:
-            ev[4].record(stream)
+        ev[4].record(stream)
 
     K, W = args.steps, args.warmup
     for _ in range(W):
@@ -229,29 +238,40 @@ def run_ours(args):
     if fa.device_status() != 0:
         raise RuntimeError("kernel status word set during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    kp = max(2, K // 2)  # per-kernel steps on each side of the timed ones (power state brackets them)
+    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(2 * kp)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(torch, world)
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
+        for i in range(kp):
+            step_per_kernel(evk[i])
+        torch.cuda.synchronize(dev)
+        barrier(torch, world)
         t0.record(stream)
         for i in range(K):
             step(evs[i])
         t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(torch, world)
+        for i in range(kp, 2 * kp):
+            step_per_kernel(evk[i])
         torch.cuda.synchronize(dev)
     barrier(torch, world)
     ms = t0.elapsed_time(t1)
     ms_max = max_over_ranks(torch, world, ms)
     if fa.device_status() != 0:
         raise RuntimeError("kernel status word set during the timed region")
-    per = {name: statistics.fmean(e[j].elapsed_time(e[j + 1]) for e in evs)
+    fwd_ms_step = statistics.fmean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in evs)
+    per = {name: statistics.fmean(e[j].elapsed_time(e[j + 1]) for e in evk)
            for j, name in enumerate(("fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"))}
 
     F = attn_flops(B, Hq, N, N, d, True)
     ms_step = ms_max / K
     value = job_throughput(world, F * 3.5, ms_step)
-    fwd_tflops = F / (per["fwd"] * 1e-3) / 1e12
-    bwd_ms = per["bwd_preprocess"] + per["bwd_dkdv"] + per["bwd_dq"]
+    fwd_tflops = F / (fwd_ms_step * 1e-3) / 1e12
     bwd_tflops = 2.5 * F / (bwd_ms * 1e-3) / 1e12
 
     # roofline of the kernel with the largest share of the step
@@ -295,13 +315,16 @@ def run_ours(args):
                    "global_batch": B * world, "seq_len": N, "parallelism": f"replicas x{world} (weak)",
                    "l2": f"no flush: each step touches {touched / 2**20:.0f} MiB (> 126 MB L2 at N=8192)",
                    "flops_convention": "fwd 4*B*Hq*N*N*d/2 (causal); bwd 2.5x fwd"},
-        "parts": {"fwd_ms": round(per["fwd"], 4), "fwd_tflops": round(fwd_tflops, 1),
+        "parts": {"fwd_ms": round(fwd_ms_step, 4), "fwd_tflops": round(fwd_tflops, 1),
                   "fwd_frac_of_datasheet_2250": round(fwd_tflops / DENSE_BF16_DATASHEET_TFLOPS, 4),
                   "fwd_frac_of_measured": round(fwd_tflops / peak, 4),
                   "bwd_ms": round(bwd_ms, 4), "bwd_tflops": round(bwd_tflops, 1),
                   "bwd_frac_of_datasheet_2250": round(bwd_tflops / DENSE_BF16_DATASHEET_TFLOPS, 4),
                   "bwd_frac_of_measured": round(bwd_tflops / peak, 4),
-                  "per_kernel_ms": {kk: round(vv, 4) for kk, vv in per.items()}},
+                  "per_kernel_ms": {kk: round(vv, 4) for kk, vv in per.items()},
+                  "per_kernel_note": "K/2 steps before and K/2 after the timed ones, one entry point per "
+                                     "launch with an event between launches (the timed steps call fa_bwd, whose "
+                                     "dQ launch overlaps the end of dK/dV)"},
         "decode": decode,
         "fp8": fp8,
         "blocksparse": sparse,
@@ -649,29 +672,43 @@ def run_long_context(args, torch, fa, _lib, workloads, dev, stream, world, peaks
     dt = _lib.FA_BF16
     bargs = [t.data_ptr() for t in (q, k, v, o, do, lse, dq, dk, dv, ws)] + [B, Hq, Hkv, N, N, d, 1, w.scale, dt, sh]
 
-    def step(ev=None):
-        if ev:
-            ev[0].record(stream)
+    def fwd():
         _lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, N, d, 1,
                     w.scale, dt, sh)
+
+    def step(ev=None):  # as a user runs it: fa_fwd, then the one-call fa_bwd
+        if ev:
+            ev[0].record(stream)
+        fwd()
         if ev:
             ev[1].record(stream)
-        _lib.fa_bwd_preprocess(*bargs)
+        _lib.fa_bwd(*bargs)
         if ev:
             ev[2].record(stream)
+
+    def step_per_kernel(ev):  # one entry point per launch, an event between launches
+        ev[0].record(stream)
+        fwd()
+        ev[1].record(stream)
+        _lib.fa_bwd_preprocess(*bargs)
+        ev[2].record(stream)
         _lib.fa_bwd_dkdv(*bargs)
-        if ev:
-            ev[3].record(stream)
+        ev[3].record(stream)
         _lib.fa_bwd_dq(*bargs)
-        if ev:
-            ev[4].record(stream)
+        ev[4].record(stream)
 
     for _ in range(args.warmup):
         step()
     K = max(3, args.steps // 2)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    kp = max(2, K // 2)  # per-kernel steps on each side of the timed ones
+    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(2 * kp)]
     barrier(torch, world)
     torch.cuda.synchronize(dev)
+    for i in range(kp):
+        step_per_kernel(evk[i])
+    torch.cuda.synchronize(dev)
+    barrier(torch, world)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(K):
@@ -679,25 +716,30 @@ def run_long_context(args, torch, fa, _lib, workloads, dev, stream, world, peaks
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(torch, world)
+    for i in range(kp, 2 * kp):
+        step_per_kernel(evk[i])
+    torch.cuda.synchronize(dev)
+    barrier(torch, world)
     if fa.device_status() != 0:
         raise RuntimeError("kernel status word set during the long-context section")
     ms_total = t0.elapsed_time(t1)
     ms = max_over_ranks(torch, world, ms_total) / K
-    per = {name: statistics.fmean(e[j].elapsed_time(e[j + 1]) for e in evs)
+    per = {name: statistics.fmean(e[j].elapsed_time(e[j + 1]) for e in evk)
            for j, name in enumerate(("fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"))}
     F = attn_flops(B, Hq, N, N, d, True)
-    bwd_ms = per["bwd_preprocess"] + per["bwd_dkdv"] + per["bwd_dq"]
+    fwd_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in evs)
     peak, key = _peak_for(peaks, ms_total)
     kflops = {"fwd": F, "bwd_dkdv": 2.0 * F, "bwd_dq": 1.5 * F}
     dom = max(kflops, key=lambda n: per[n])
     kname = {"fwd": "fwd_sm100_kernel", "bwd_dkdv": "bwd_dkdv_sm100_kernel", "bwd_dq": "bwd_dq_sm100_kernel"}[dom]
     ach = kflops[dom] / (per[dom] * 1e-3) / 1e12
-    fwd_t, bwd_t = F / (per["fwd"] * 1e-3) / 1e12, 2.5 * F / (bwd_ms * 1e-3) / 1e12
+    fwd_t, bwd_t = F / (fwd_ms * 1e-3) / 1e12, 2.5 * F / (bwd_ms * 1e-3) / 1e12
     traffic8192 = traffic_for(kname)
     traffic8192 = None if traffic8192 is None else int(traffic8192 * N / 8192)
     return {"workload": f"long-context GQA step: fwd+bwd, B={B} Hq={Hq} Hkv={Hkv} Nq=Nk={N} d={d} causal bf16",
             "ms_per_step": round(ms, 4), "value": round(world * 3.5 * F / (ms * 1e-3) / 1e12, 1), "unit": "TFLOP/s",
-            "fwd_ms": round(per["fwd"], 4), "fwd_tflops": round(fwd_t, 1),
+            "fwd_ms": round(fwd_ms, 4), "fwd_tflops": round(fwd_t, 1),
             "fwd_frac_of_datasheet_2250": round(fwd_t / DENSE_BF16_DATASHEET_TFLOPS, 4),
             "bwd_ms": round(bwd_ms, 4), "bwd_tflops": round(bwd_t, 1),
             "bwd_frac_of_datasheet_2250": round(bwd_t / DENSE_BF16_DATASHEET_TFLOPS, 4),

@@ -234,6 +234,9 @@ __global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
   const int nq = (p.Nq + kT - 1) / kT;
   const int per_head = nq - mstart;
   const int nt = G * per_head;  // query tiles this CTA visits
+  // the dQ kernel, launched next on the stream as a programmatic dependent, reads none of this
+  // kernel's outputs: let its CTAs start on SMs this grid frees (its last CTA waits for this grid)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (tid == 0) {
     for (int i = 0; i < L::kNumBars; ++i)
@@ -815,6 +818,11 @@ __global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
+  // launched as a programmatic dependent of the dK/dV kernel: the grid must not complete before
+  // that kernel has (later work on the stream waits only for this grid), so the last CTA waits
+  // for it; without that launch attribute the wait returns at once
+  if (blockIdx.x == gridDim.x - 1 && blockIdx.y == gridDim.y - 1 && blockIdx.z == gridDim.z - 1)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -883,9 +891,19 @@ cudaError_t launch_dq(const BwdArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   if (drop && !split_fits(kern)) return cudaErrorInvalidConfiguration;
   dim3 grid(a.Hq, (a.Nq + kT - 1) / kT, a.B);
-  kern<<<grid, drop ? kThreadsDrop : kThreads, smem, s>>>(m.q, m.k, m.v, m.dO, m.dq,
-                                                          params(a, a.dq, nullptr, a.acc_q, nullptr));
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(drop ? kThreadsDrop : kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr{};
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  if (a.after_dkdv) {  // the previous launch on the stream is this backward's dK/dV kernel
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, m.q, m.k, m.v, m.dO, m.dq, params(a, a.dq, nullptr, a.acc_q, nullptr));
 }
 
 }  // namespace

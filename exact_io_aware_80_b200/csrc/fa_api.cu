@@ -279,6 +279,7 @@ static fa_status bwd_run(int steps, const void* q, const void* k, const void* v,
   cudaError_t e = cudaSuccess;
   if (pre) e = fa::launch_bwd_preprocess(a, s);
   if (e == cudaSuccess && dkdv) e = fa::launch_bwd_dkdv_sm100(a, s);
+  a.after_dkdv = dkdv ? 1 : 0;
   if (e == cudaSuccess && dqs) e = fa::launch_bwd_dq_sm100(a, s);
   return from_cuda(e);
 }
@@ -455,5 +456,6 @@ fa_status fa_bwd_accumulate(const void* q, const void* k, const void* v, const v
   fa::BwdArgs qa = a;
   qa.acc_q = dq_acc;
   qa.acc_init = (init & 1) ? 1 : 0;
+  qa.after_dkdv = 1;
   return from_cuda(fa::launch_bwd_dq_sm100(qa, s));
 }

@@ -58,6 +58,9 @@ struct BwdArgs {
   float* acc_k = nullptr;
   float* acc_v = nullptr;
   int acc_init = 0;
+  // the dQ launch directly follows this backward's dK/dV launch on the same stream: it may
+  // start as a programmatic dependent (the two kernels share inputs, not outputs)
+  int after_dkdv = 0;
 };
 
 struct DecodeArgs {

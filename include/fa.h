@@ -85,7 +85,10 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq);
  * must hold fa_bwd_workspace_bytes(B, Hq, Nq) bytes (device, 16-byte aligned).
  * No atomics: dK/dV and dQ come from separate kernels, so the result is
  * bitwise reproducible (the deterministic mode of the smithlab guide's
- * recommendation table).
+ * recommendation table).  The dQ kernel is launched as a programmatic
+ * dependent of the dK/dV kernel and may start on SMs that dK/dV has released;
+ * the call still behaves as one stream operation: work enqueued after it on
+ * `stream` starts only after every gradient is written.
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                  const float* lse, void* dq, void* dk, void* dv, void* workspace,
