@@ -280,6 +280,9 @@ __global__ void __launch_bounds__(kRows, 3) quant_kernel(QuantJobs jobs, const f
   if (signs)
     for (int i = threadIdx.x; i < D; i += kRows) s_signs[i] = signs[i];
   const float* sg = signs ? s_signs : nullptr;  // visible to every thread after the loop's first barrier
+  // V's encode, launched next as a programmatic dependent, may stage its V rows meanwhile; it
+  // waits for this grid before it reads the block maxima
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   long id = blockIdx.x;
   if (id < total) issue_block<T, D>(jobs, block_ref(jobs, id, B), stage[0]);
   cp_async_commit();
@@ -347,7 +350,10 @@ __global__ void __launch_bounds__(kRows) v_quant_kernel(const T* __restrict__ v,
   __shared__ float red[4];
   issue_rows<T, D>(v, st, Nk, H, b, h, j * kRows);
   cp_async_commit();
-  // the head's amax over its block maxima, while the block's copies are in flight
+  // the head's amax over its block maxima, while the block's copies are in flight.  Launched as a
+  // programmatic dependent of the kernel that wrote them: wait for that grid first (without the
+  // launch attribute the wait returns at once)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   float amax = 0.f;
   const float* ph = part + ((long)b * H + h) * nb;
   for (int i = threadIdx.x; i < nb; i += kRows) amax = fmaxf(amax, ph[i]);
@@ -398,13 +404,22 @@ cudaError_t launch_jobs(const QuantJobs& jobs, const float* signs, int B, cudaSt
 template <typename T, int D>
 cudaError_t launch_v_quant(const void* v, const float* part, void* v8t, float* scale, int B, int H, int Nk,
                            int* status, cudaStream_t s) {
-  dim3 grid((Nk + kRows - 1) / kRows, H, B);
   constexpr int smem = VQuantSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(v_quant_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  v_quant_kernel<T, D><<<grid, kRows, smem, s>>>(static_cast<const T*>(v), part, static_cast<uint8_t*>(v8t), scale, Nk,
-                                                H, (Nk + 15) / 16 * 16, status);
-  return cudaGetLastError();
+  // always launched right after the quant_kernel launch that writes `part`, on the same stream
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((Nk + kRows - 1) / kRows, H, B);
+  cfg.blockDim = dim3(kRows);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr{};
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, v_quant_kernel<T, D>, static_cast<const T*>(v), part, static_cast<uint8_t*>(v8t),
+                            scale, Nk, H, (Nk + 15) / 16 * 16, status);
 }
 
 template <int D>
