@@ -239,23 +239,24 @@ def run_ours(args):
         raise RuntimeError("kernel status word set during warm-up")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    kp = max(2, K // 2)  # per-kernel steps on each side of the timed ones (power state brackets them)
-    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(2 * kp)]
+    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(torch, world)
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
-        for i in range(kp):
-            step_per_kernel(evk[i])
-        torch.cuda.synchronize(dev)
-        barrier(torch, world)
         t0.record(stream)
         for i in range(K):
             step(evs[i])
         t1.record(stream)
         torch.cuda.synchronize(dev)
         barrier(torch, world)
-        for i in range(kp, 2 * kp):
+        # per-kernel pass under the same starting conditions as the timed steps: the GPU idles
+        # briefly (its power management recovers from the timed steps), then W warm-up and K
+        # measured steps
+        time.sleep(0.5)
+        for _ in range(W):
+            step()
+        for i in range(K):
             step_per_kernel(evk[i])
         torch.cuda.synchronize(dev)
     barrier(torch, world)
@@ -322,9 +323,9 @@ def run_ours(args):
                   "bwd_frac_of_datasheet_2250": round(bwd_tflops / DENSE_BF16_DATASHEET_TFLOPS, 4),
                   "bwd_frac_of_measured": round(bwd_tflops / peak, 4),
                   "per_kernel_ms": {kk: round(vv, 4) for kk, vv in per.items()},
-                  "per_kernel_note": "K/2 steps before and K/2 after the timed ones, one entry point per "
-                                     "launch with an event between launches (the timed steps call fa_bwd, whose "
-                                     "dQ launch overlaps the end of dK/dV)"},
+                  "per_kernel_note": "K more steps after a 0.5 s idle and W warm-up steps, one entry point "
+                                     "per launch with an event between launches (the timed steps call fa_bwd, "
+                                     "whose dQ launch overlaps the end of dK/dV)"},
         "decode": decode,
         "fp8": fp8,
         "blocksparse": sparse,
@@ -701,14 +702,9 @@ def run_long_context(args, torch, fa, _lib, workloads, dev, stream, world, peaks
         step()
     K = max(3, args.steps // 2)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    kp = max(2, K // 2)  # per-kernel steps on each side of the timed ones
-    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(2 * kp)]
+    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
     barrier(torch, world)
     torch.cuda.synchronize(dev)
-    for i in range(kp):
-        step_per_kernel(evk[i])
-    torch.cuda.synchronize(dev)
-    barrier(torch, world)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(K):
@@ -716,7 +712,10 @@ def run_long_context(args, torch, fa, _lib, workloads, dev, stream, world, peaks
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(torch, world)
-    for i in range(kp, 2 * kp):
+    time.sleep(0.5)  # per-kernel pass from the same starting conditions as the timed steps
+    for _ in range(args.warmup):
+        step()
+    for i in range(K):
         step_per_kernel(evk[i])
     torch.cuda.synchronize(dev)
     barrier(torch, world)

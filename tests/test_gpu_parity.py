@@ -303,6 +303,42 @@ def test_bitwise_determinism(fa):
     assert fa.device_status() == 0
 
 
+def test_one_call_backward_equals_separate_launches_and_orders_the_stream(fa):
+    """Inside fa_bwd the dQ kernel is a programmatic dependent of dK/dV (it may start while dK/dV
+    runs).  Its gradients must equal those of the three entry points called one at a time, and
+    work enqueued on the stream right after fa_bwd must see every gradient complete: the sums
+    taken there, before any host synchronisation, must equal the sums of the final tensors."""
+    from exact_io_aware_80_b200 import _lib
+    B, Hq, Hkv, N, d = 1, 16, 4, 4096, 128  # dK/dV: 128 CTAs; dQ: 512 CTAs
+    q, k, v, do = [t.cuda() for t in workloads.make_inputs(B, Hq, Hkv, N, N, d, torch.bfloat16, seed_base=51,
+                                                           with_do=True)]
+    o, lse = fa.attention_fwd(q, k, v, True)
+    ws = torch.empty(fa.fa_bwd_workspace_bytes(B, Hq, N), device="cuda", dtype=torch.uint8)
+    grads = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
+    st = torch.cuda.current_stream().cuda_stream
+    args = [t.data_ptr() for t in (q, k, v, o, do, lse, *grads, ws)] + [B, Hq, Hkv, N, N, d, 1, 1.0 / math.sqrt(d),
+                                                                       _lib.FA_BF16, st]
+    _lib.fa_bwd_preprocess(*args)
+    _lib.fa_bwd_dkdv(*args)
+    _lib.fa_bwd_dq(*args)
+    torch.cuda.synchronize()
+    ref = [g.clone() for g in grads]
+    sums = []
+    for _ in range(12):
+        for g in grads:
+            g.zero_()
+        _lib.fa_bwd(*args)
+        sums.append([g.float().sum() for g in grads])  # enqueued behind fa_bwd, no host sync
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    for g, r in zip(grads, ref):
+        assert torch.equal(g, r)
+    final = [g.float().sum() for g in grads]
+    for s3 in sums:
+        for a, b in zip(s3, final):
+            assert torch.equal(a, b)
+
+
 def test_watchdog_times_out_cleanly_and_context_survives(fa):
     """A bounded wait on a barrier nothing arrives on reports FA_ERR_TIMEOUT
     through the status word (no trap, no hang), which then reads clean again,
