@@ -57,6 +57,17 @@ constexpr int kThreads = 192;  // warps 0-3 elementwise, 4 TMA, 5 MMA
 constexpr int kThreadsDrop = 384;
 constexpr int kRegsElem = 256, kRegsCtrl = 104, kRegsRng = 104;
 static_assert(128 * (kRegsElem + kRegsCtrl + kRegsRng) <= kThreadsDrop * 168, "register split exceeds the launch");
+// Of every eight column pairs, how many exponentials take the FMA pipe (exp2_fma2) instead of
+// ex2.approx, without and with dropout (whose keep-bit generator shares the multiply pipe, so
+// there every exponential goes to ex2.approx: 2.91 -> 2.87 ms for the dropout backward at N=8192).
+#ifndef FA_BWD_EXP2_EIGHTHS
+#define FA_BWD_EXP2_EIGHTHS 2
+#endif
+#ifndef FA_BWD_DROP_EXP2_EIGHTHS
+#define FA_BWD_DROP_EXP2_EIGHTHS 0
+#endif
+template <bool DROP>
+constexpr int kExp8 = DROP ? FA_BWD_DROP_EXP2_EIGHTHS : FA_BWD_EXP2_EIGHTHS;
 constexpr int kWarpLoad = 4;
 constexpr int kWarpMma = 5;
 constexpr int kPanel = 128 * 128;  // [128 rows][64 cols] 16-bit panel, bytes
@@ -447,7 +458,8 @@ __global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
       const float2 c2 = make_float2(c, c);
 #pragma unroll
       for (int cc = 0; cc < kT; cc += 2) {
-        const float2 x = exp2_pair(__ffma2_rn(make_float2(pv[cc], pv[cc + 1]), c2, nl2[cc >> 1]), cc >> 1);
+        const float2 x =
+            exp2_pair8<kExp8<DROP>>(__ffma2_rn(make_float2(pv[cc], pv[cc + 1]), c2, nl2[cc >> 1]), cc >> 1);
         pv[cc] = x.x;
         pv[cc + 1] = x.y;
       }
@@ -754,7 +766,7 @@ __global__ void __launch_bounds__(DROP ? kThreadsDrop : kThreads, 1)
       const float2 c2 = make_float2(c, c), nl2 = make_float2(nlse2, nlse2);
 #pragma unroll
       for (int cc = 0; cc < kT; cc += 2) {
-        const float2 x = exp2_pair(__ffma2_rn(make_float2(pv[cc], pv[cc + 1]), c2, nl2), cc >> 1);
+        const float2 x = exp2_pair8<kExp8<DROP>>(__ffma2_rn(make_float2(pv[cc], pv[cc + 1]), c2, nl2), cc >> 1);
         pv[cc] = x.x;
         pv[cc + 1] = x.y;
       }

@@ -82,12 +82,16 @@ constexpr int kThreads = 384;
 constexpr int kRegsSoftmax = 200;
 constexpr int kRegsControl = 104;
 // Of every eight column pairs of a score block, how many take the FMA-pipe exponential
-// (exp2_fma2) instead of ex2.approx, with 16-bit and with FP8 operands.
+// (exp2_fma2) instead of ex2.approx: 16-bit operands, FP8 operands, 16-bit with dropout (whose
+// Philox multiplies share the FMA pipe).
 #ifndef FA_FWD_EXP2_EIGHTHS
 #define FA_FWD_EXP2_EIGHTHS 2
 #endif
 #ifndef FA_FWD_F8_EXP2_EIGHTHS
 #define FA_FWD_F8_EXP2_EIGHTHS 2
+#endif
+#ifndef FA_FWD_DROP_EXP2_EIGHTHS
+#define FA_FWD_DROP_EXP2_EIGHTHS 2
 #endif
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * 168, "register split exceeds the launch");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when m grows by more than 2^8
@@ -220,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, Params p) {
   using L = Smem<D, F8>;
-  constexpr int kExpFma8 = F8 ? FA_FWD_F8_EXP2_EIGHTHS : FA_FWD_EXP2_EIGHTHS;
+  constexpr int kExpFma8 = F8 ? FA_FWD_F8_EXP2_EIGHTHS : DROP ? FA_FWD_DROP_EXP2_EIGHTHS : FA_FWD_EXP2_EIGHTHS;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
