@@ -278,22 +278,10 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
                      __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
-// Of every four column pairs, how many take exp2_fma2 instead of ex2.approx.
-#ifndef FA_EXP2_FMA_PAIRS
-#define FA_EXP2_FMA_PAIRS 1
-#endif
-constexpr int kExp2FmaPairs = FA_EXP2_FMA_PAIRS;
-
-// 2^x for a pair of columns, routed by the pair's index (a constant once the
-// caller's loop is unrolled, so the branch folds away).
-__device__ __forceinline__ float2 exp2_pair(float2 x, int pair) {
-  if ((pair & 3) >= 4 - kExp2FmaPairs) return exp2_fma2(x);
-  return make_float2(ex2(x.x), ex2(x.y));
-}
-
-// The same with the share in eighths: K of every 8 consecutive column pairs, spread evenly
-// (pair p takes the FMA form when floor((p + 1) K / 8) > floor(p K / 8); K = 2 picks pairs
-// 3 and 7 of every 8, as exp2_pair with one pair in four).
+// 2^x for a pair of columns, routed by the pair's index (a constant once the caller's loop is
+// unrolled, so the branch folds away): K of every 8 consecutive column pairs, spread evenly, take
+// exp2_fma2, the others ex2.approx (pair p takes the FMA form when floor((p + 1) K / 8) >
+// floor(p K / 8); K = 2 picks pairs 3 and 7 of every 8).
 template <int K>
 __device__ __forceinline__ float2 exp2_pair8(float2 x, int pair) {
   if (((pair + 1) * K) / 8 != (pair * K) / 8) return exp2_fma2(x);
