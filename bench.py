@@ -4,8 +4,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 A step is one GQA training step of attention: forward then backward on
-B=1, Hq=32, Hkv=8, N=8192, d=128, causal, bf16 (fwd kernel, then the three
-backward launches: D preprocess, dK/dV, dQ).  ``value`` is whole-job
+B=1, Hq=32, Hkv=8, N=8192, d=128, causal, bf16, called as a user calls it
+(fa_fwd, then fa_bwd: D preprocess, dK/dV, and dQ as a programmatic dependent
+of dK/dV); per-kernel durations for the roofline come from a second pass of
+the same steps with one entry point per launch.  ``value`` is whole-job
 fwd+bwd TFLOP/s with the inputs resident in HBM, FLOPs counted as
 4 B Hq Nq Nk d / 2 for the causal forward and 2.5x that for the backward.
 The split-KV decode workload (B=64, Hq=32, Hkv=8, Nk_max=32768 with a ragged
